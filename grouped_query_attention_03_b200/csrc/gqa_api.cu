@@ -1,0 +1,431 @@
+// gqa_api.cu -- the C ABI declared in include/gqa.h.
+//
+// Host-side validation (the checked constructor conditions of "Share
+// key/value heads and make context explicit", section "Give each query head
+// an explicit shared KV head": positive head counts and width, Hq divisible
+// by Hkv; the refused zero window of "Intersect the window ..."; checked size
+// products as in its incremental path), then kernel launches on the caller's
+// stream.  Nothing here allocates device memory.
+#include <algorithm>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/gqa.h"
+#include "append.cuh"
+#include "common.cuh"
+#include "decode_splitk.cuh"
+#include "prefill_tc.cuh"
+#include "simt.cuh"
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kMaxDecodeCtas = 1024;  // workspace is sized for this many
+constexpr int kDecodeMinRows = 128;   // rows below which a CTA is not split
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0;
+};
+
+gqa_status device_info(DeviceInfo *out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!have[dev]) {
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor,
+                               dev) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    cache[dev] = d;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  return out->major == 10 ? GQA_OK : GQA_ERR_DEVICE;
+}
+
+// a*b*... in int64 with overflow detection (all factors >= 0).
+bool mul_ok(int64_t *acc, int64_t f) {
+  if (f < 0) return false;
+  if (f != 0 && *acc > INT64_MAX / f) return false;
+  *acc *= f;
+  return true;
+}
+
+bool elems(int64_t *out, std::initializer_list<int64_t> dims) {
+  int64_t acc = 1;
+  for (int64_t d : dims)
+    if (!mul_ok(&acc, d)) return false;
+  *out = acc;
+  return true;
+}
+
+bool aligned16(const void *p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+gqa_status check_heads(int Hq, int Hkv, int d) {
+  if (Hq <= 0 || Hkv <= 0 || d <= 0) return GQA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return GQA_ERR_GROUPS;
+  return GQA_OK;
+}
+
+gqa_status check_window(int window) {
+  return (window == 0 || window < -1) ? GQA_ERR_WINDOW : GQA_OK;
+}
+
+gqa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// ------------------------------------------------------------ decode plan
+struct DecPlan {
+  int R = 1;     // heads stacked per CTA lane (power of two, <= 8)
+  int nsub = 1;  // sub-groups per KV head
+  int VL = 1;    // virtual lanes per batch row
+};
+
+DecPlan decode_plan(int Hq, int Hkv) {
+  DecPlan p;
+  const int r = Hq / Hkv;
+  p.R = r >= 8 ? 8 : next_pow2(r);
+  p.nsub = (r + p.R - 1) / p.R;
+  p.VL = Hkv * p.nsub;
+  return p;
+}
+
+struct DecLayout {
+  size_t hdr = 0, lane_start = 0, ml = 0, acc = 0, total = 0;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
+  const DecPlan pl = decode_plan(Hq, Hkv);
+  int64_t lanes, slots, ml_elems, acc_elems;
+  if (!elems(&lanes, {B, pl.VL})) return false;
+  slots = lanes + kMaxDecodeCtas;
+  if (!elems(&ml_elems, {slots, pl.R})) return false;
+  if (!elems(&acc_elems, {slots, pl.R, d})) return false;
+  if (acc_elems > INT64_MAX / 8) return false;
+  L->hdr = 0;
+  L->lane_start = round256(sizeof(gqa::dec::WsHdr));
+  L->ml = L->lane_start + round256((size_t)lanes * sizeof(long long));
+  L->acc = L->ml + round256((size_t)ml_elems * sizeof(float2));
+  L->total = L->acc + round256((size_t)acc_elems * sizeof(float));
+  return true;
+}
+
+bool splitk_supported(gqa_dtype dtype, int d) {
+  return dtype == GQA_BF16 && (d == 64 || d == 128);
+}
+
+template <int D, int R>
+gqa_status launch_splitk(const gqa::dec::Params &p, int sms, cudaStream_t st) {
+  using K = gqa::dec::Cfg<D, R>;
+  const int smem = K::STAGES * K::STAGE_BYTES;
+  static bool attr_done = false;  // per instantiation; benign race
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(gqa::dec::split_kernel<D, R>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    attr_done = true;
+  }
+  const int grid = std::min(kMaxDecodeCtas, 2 * sms);
+  gqa::dec::split_kernel<D, R><<<grid, gqa::dec::kThreads, smem, st>>>(p);
+  if (launch_status() != GQA_OK) return GQA_ERR_CUDA;
+  gqa::dec::merge_kernel<D, R><<<dim3(p.VL, p.B), 128, 0, st>>>(p);
+  return launch_status();
+}
+
+template <int D>
+gqa_status dispatch_splitk_R(int R, const gqa::dec::Params &p, int sms,
+                             cudaStream_t st) {
+  switch (R) {
+    case 1: return launch_splitk<D, 1>(p, sms, st);
+    case 2: return launch_splitk<D, 2>(p, sms, st);
+    case 4: return launch_splitk<D, 4>(p, sms, st);
+    case 8: return launch_splitk<D, 8>(p, sms, st);
+  }
+  return GQA_ERR_UNSUPPORTED;
+}
+
+template <typename T>
+gqa_status launch_simt_prefill(const void *q, const void *k, const void *v,
+                               void *o, const int32_t *lens, int B, int Hq,
+                               int Hkv, int T_len, int d, int window,
+                               float scale_log2, int32_t *status,
+                               cudaStream_t st) {
+  const dim3 grid((T_len + 3) / 4, Hq, B);
+  const int nf = (d + 31) / 32;
+#define GQA_PF(NF)                                                        \
+  gqa::prefill_simt_kernel<T, NF><<<grid, 128, 0, st>>>(                  \
+      (const T *)q, (const T *)k, (const T *)v, (T *)o, lens, Hq, Hkv,    \
+      T_len, d, window, scale_log2, status)
+  switch (nf) {
+    case 1: GQA_PF(1); break;
+    case 2: GQA_PF(2); break;
+    case 3: GQA_PF(3); break;
+    case 4: GQA_PF(4); break;
+    case 5: GQA_PF(5); break;
+    case 6: GQA_PF(6); break;
+    case 7: GQA_PF(7); break;
+    case 8: GQA_PF(8); break;
+    default: return GQA_ERR_UNSUPPORTED;
+  }
+#undef GQA_PF
+  return launch_status();
+}
+
+template <typename T>
+gqa_status launch_simt_decode(const void *q, const void *kc, const void *vc,
+                              void *o, const int32_t *lens, int B, int Hq,
+                              int Hkv, int C, int d, int window,
+                              float scale_log2, int32_t *status,
+                              cudaStream_t st) {
+  const dim3 grid(Hq, B);
+  const int nf = (d + 31) / 32;
+#define GQA_DC(NF)                                                         \
+  gqa::decode_simt_kernel<T, NF><<<grid, 32, 0, st>>>(                     \
+      (const T *)q, (const T *)kc, (const T *)vc, (T *)o, lens, B, Hq, Hkv, \
+      C, d, window, scale_log2, status)
+  switch (nf) {
+    case 1: GQA_DC(1); break;
+    case 2: GQA_DC(2); break;
+    case 3: GQA_DC(3); break;
+    case 4: GQA_DC(4); break;
+    case 5: GQA_DC(5); break;
+    case 6: GQA_DC(6); break;
+    case 7: GQA_DC(7); break;
+    case 8: GQA_DC(8); break;
+    default: return GQA_ERR_UNSUPPORTED;
+  }
+#undef GQA_DC
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gqa_version(void) { return "0.1.0"; }
+
+const char *gqa_status_string(gqa_status s) {
+  switch (s) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_NULL: return "a required pointer is NULL";
+    case GQA_ERR_SHAPE: return "a size is negative or a head count/width is not positive";
+    case GQA_ERR_GROUPS: return "query heads are not a multiple of KV heads";
+    case GQA_ERR_WINDOW: return "window must be -1 (none) or positive";
+    case GQA_ERR_CAPACITY: return "a sequence length is outside [0, capacity]";
+    case GQA_ERR_OVERFLOW: return "an element count overflows";
+    case GQA_ERR_UNSUPPORTED: return "head width, dtype, alignment or grid size not supported";
+    case GQA_ERR_WORKSPACE: return "workspace missing or too small";
+    case GQA_ERR_CUDA: return "CUDA runtime error";
+    case GQA_ERR_DEVICE: return "current device is not an sm_100 GPU";
+    case GQA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+  }
+  return "unknown status";
+}
+
+int gqa_kv_head_for_query(int h, int Hq, int Hkv) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return -1;
+  if (h < 0 || h >= Hq) return -1;
+  return h / (Hq / Hkv);
+}
+
+int gqa_window_start(int t, int window) {
+  if (t < 0 || window == 0 || window < -1) return -1;
+  if (window < 0) return 0;
+  return t > window - 1 ? t - (window - 1) : 0;
+}
+
+uint64_t gqa_cache_bytes(int64_t L, int64_t B, int64_t T, int64_t Hkv,
+                         int64_t d, int64_t elem_bytes) {
+  const int64_t f[6] = {L, B, T, Hkv, d, elem_bytes};
+  uint64_t acc = 2;
+  for (int i = 0; i < 6; ++i) {
+    if (f[i] < 0) return 0;
+    const uint64_t x = (uint64_t)f[i];
+    if (x != 0 && acc > UINT64_MAX / x) return 0;
+    acc *= x;
+  }
+  return acc;
+}
+
+gqa_status gqa_prefill(gqa_dtype dtype, const void *q, const void *k,
+                       const void *v, void *o, const int32_t *seq_lens, int B,
+                       int Hq, int Hkv, int T, int d, int window, float scale,
+                       int32_t *dev_status, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  if (B < 0 || T < 0) return GQA_ERR_SHAPE;
+  gqa_status s = check_heads(Hq, Hkv, d);
+  if (s != GQA_OK) return s;
+  if ((s = check_window(window)) != GQA_OK) return s;
+  int64_t nq, nk;
+  if (!elems(&nq, {B, Hq, T, d}) || !elems(&nk, {B, Hkv, T, d}) ||
+      nq > INT64_MAX / 4)
+    return GQA_ERR_OVERFLOW;
+  if (B == 0 || T == 0) return GQA_OK;
+  if (!q || !k || !v || !o) return GQA_ERR_NULL;
+  if (d > GQA_MAX_HEAD_DIM) return GQA_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if ((s = device_info(&di)) != GQA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float scale_log2 = scale * gqa::kLog2e;
+  if (dtype == GQA_BF16 && gqa::pf::supported(d) && aligned16(q) &&
+      aligned16(k) && aligned16(v) && aligned16(o)) {
+    return gqa::pf::launch(q, k, v, o, seq_lens, B, Hq, Hkv, T, d, window,
+                           scale_log2, dev_status, di.sms, st);
+  }
+  if (Hq > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
+  if (dtype == GQA_F32)
+    return launch_simt_prefill<float>(q, k, v, o, seq_lens, B, Hq, Hkv, T, d,
+                                      window, scale_log2, dev_status, st);
+  return launch_simt_prefill<bf16>(q, k, v, o, seq_lens, B, Hq, Hkv, T, d,
+                                   window, scale_log2, dev_status, st);
+}
+
+size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,
+                                  int C, int d) {
+  if (B < 0 || C < 0 || check_heads(Hq, Hkv, d) != GQA_OK) return 0;
+  if (!splitk_supported(dtype, d)) return 0;
+  DecLayout L;
+  if (!decode_layout(B, Hq, Hkv, d, &L)) return 0;
+  return L.total;
+}
+
+gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
+                      const void *v_cache, void *o, const int32_t *seq_lens,
+                      int B, int Hq, int Hkv, int C, int d, int window,
+                      float scale, void *workspace, size_t workspace_bytes,
+                      int32_t *dev_status, gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  if (B < 0 || C < 0) return GQA_ERR_SHAPE;
+  gqa_status s = check_heads(Hq, Hkv, d);
+  if (s != GQA_OK) return s;
+  if ((s = check_window(window)) != GQA_OK) return s;
+  int64_t nq, nc;
+  if (!elems(&nq, {B, Hq, d}) || !elems(&nc, {B, Hkv, C, d}) ||
+      nc > INT64_MAX / 4)
+    return GQA_ERR_OVERFLOW;
+  if (B == 0) return GQA_OK;
+  if (!q || !k_cache || !v_cache || !o || !seq_lens || !dev_status)
+    return GQA_ERR_NULL;
+  if (d > GQA_MAX_HEAD_DIM) return GQA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float scale_log2 = scale * gqa::kLog2e;
+  const bool aligned = aligned16(q) && aligned16(k_cache) &&
+                       aligned16(v_cache) && aligned16(o);
+  DeviceInfo di;
+  if (splitk_supported(dtype, d) && aligned) {
+    DecLayout L;
+    if (!decode_layout(B, Hq, Hkv, d, &L)) return GQA_ERR_OVERFLOW;
+    if (!workspace || workspace_bytes < L.total ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return GQA_ERR_WORKSPACE;
+    const DecPlan pl = decode_plan(Hq, Hkv);
+    if (pl.VL > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
+    if ((s = device_info(&di)) != GQA_OK) return s;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    gqa::dec::Params p;
+    p.q = (const bf16 *)q;
+    p.kc = (const bf16 *)k_cache;
+    p.vc = (const bf16 *)v_cache;
+    p.o = (bf16 *)o;
+    p.seq_lens = seq_lens;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.C = C;
+    p.window = window;
+    p.scale_log2 = scale_log2;
+    p.r = Hq / Hkv;
+    p.nsub = pl.nsub;
+    p.VL = pl.VL;
+    p.min_rows = kDecodeMinRows;
+    p.hdr = reinterpret_cast<gqa::dec::WsHdr *>(ws + L.hdr);
+    p.lane_start = reinterpret_cast<long long *>(ws + L.lane_start);
+    p.ml = reinterpret_cast<float2 *>(ws + L.ml);
+    p.acc = reinterpret_cast<float *>(ws + L.acc);
+    p.status = dev_status;
+    return d == 64 ? dispatch_splitk_R<64>(pl.R, p, di.sms, st)
+                   : dispatch_splitk_R<128>(pl.R, p, di.sms, st);
+  }
+  if (Hq > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
+  if ((s = device_info(&di)) != GQA_OK) return s;
+  if (dtype == GQA_F32)
+    return launch_simt_decode<float>(q, k_cache, v_cache, o, seq_lens, B, Hq,
+                                     Hkv, C, d, window, scale_log2,
+                                     dev_status, st);
+  return launch_simt_decode<bf16>(q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv,
+                                  C, d, window, scale_log2, dev_status, st);
+}
+
+gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,
+                            const void *k_new, const void *v_new,
+                            int32_t *seq_lens, int B, int Hkv, int C, int d,
+                            int t_new, int32_t *dev_status,
+                            gqa_stream_t stream) {
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+  if (B < 0 || C < 0 || t_new < 0) return GQA_ERR_SHAPE;
+  if (Hkv <= 0 || d <= 0) return GQA_ERR_SHAPE;
+  const int esz = dtype == GQA_F32 ? 4 : 2;
+  int64_t nc, nn;
+  if (!elems(&nc, {B, Hkv, C, d, esz}) || !elems(&nn, {B, Hkv, t_new, d, esz}))
+    return GQA_ERR_OVERFLOW;
+  if (B == 0 || t_new == 0) return GQA_OK;
+  if (!k_cache || !v_cache || !k_new || !v_new || !seq_lens || !dev_status)
+    return GQA_ERR_NULL;
+  if (t_new > C) return GQA_ERR_CAPACITY;
+  DeviceInfo di;
+  gqa_status s = device_info(&di);
+  if (s != GQA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t row_bytes = (int64_t)d * esz;
+  const bool vec = row_bytes % 16 == 0 && aligned16(k_cache) &&
+                   aligned16(v_cache) && aligned16(k_new) && aligned16(v_new);
+  const int vpr = vec ? (int)(row_bytes / 16) : d;
+  const int64_t total = nn / (vec ? 16 : esz);
+  const int64_t want = (total + 255) / 256;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)di.sms * 8));
+  if (vec)
+    gqa::append_copy_kernel<uint4><<<grid, 256, 0, st>>>(
+        (uint4 *)k_cache, (uint4 *)v_cache, (const uint4 *)k_new,
+        (const uint4 *)v_new, seq_lens, B, Hkv, C, t_new, vpr, dev_status);
+  else if (esz == 4)
+    gqa::append_copy_kernel<uint32_t><<<grid, 256, 0, st>>>(
+        (uint32_t *)k_cache, (uint32_t *)v_cache, (const uint32_t *)k_new,
+        (const uint32_t *)v_new, seq_lens, B, Hkv, C, t_new, vpr, dev_status);
+  else
+    gqa::append_copy_kernel<uint16_t><<<grid, 256, 0, st>>>(
+        (uint16_t *)k_cache, (uint16_t *)v_cache, (const uint16_t *)k_new,
+        (const uint16_t *)v_new, seq_lens, B, Hkv, C, t_new, vpr, dev_status);
+  if (launch_status() != GQA_OK) return GQA_ERR_CUDA;
+  gqa::append_commit_kernel<<<1, 256, 0, st>>>(seq_lens, B, C, t_new);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,222 @@
+"""ctypes binding of the C ABI in ``include/gqa.h`` (argument marshalling only).
+
+Every computation runs in the CUDA library ``libgqa_b200.so``; this module
+checks tensor dtypes, devices and contiguity, passes raw device pointers and
+the current CUDA stream, and turns a non-zero ``gqa_status`` into
+``GQAError``.  There is no fallback: if the library is missing, every call
+raises.  PyTorch provides device memory and streams, nothing else.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+
+GQA_F32, GQA_BF16 = 0, 1
+NO_WINDOW = -1
+
+STATUS_NAMES = {
+    0: "GQA_OK", 1: "GQA_ERR_NULL", 2: "GQA_ERR_SHAPE", 3: "GQA_ERR_GROUPS",
+    4: "GQA_ERR_WINDOW", 5: "GQA_ERR_CAPACITY", 6: "GQA_ERR_OVERFLOW",
+    7: "GQA_ERR_UNSUPPORTED", 8: "GQA_ERR_WORKSPACE", 9: "GQA_ERR_CUDA",
+    10: "GQA_ERR_DEVICE", 11: "GQA_ERR_TIMEOUT",
+}
+
+# Every symbol include/gqa.h declares.
+EXPORTS = ("gqa_prefill", "gqa_decode", "gqa_decode_workspace_bytes",
+           "gqa_cache_append", "gqa_cache_bytes", "gqa_kv_head_for_query",
+           "gqa_window_start", "gqa_status_string", "gqa_version")
+
+
+class GQAError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = int(status)
+        name = STATUS_NAMES.get(self.status, str(status))
+        super().__init__(f"{what}: {name} ({_status_string(self.status)})")
+
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"CUDA library {LIB_PATH} is missing; build it with "
+                "grouped_query_attention_03_b200.build.build()")
+        _lib = _declare(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def _declare(L):
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sz, i64 = ctypes.c_size_t, ctypes.c_int64
+    L.gqa_prefill.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, vp]
+    L.gqa_prefill.restype = i32
+    L.gqa_decode.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, sz, vp, vp]
+    L.gqa_decode.restype = i32
+    L.gqa_decode_workspace_bytes.argtypes = [i32] * 6
+    L.gqa_decode_workspace_bytes.restype = sz
+    L.gqa_cache_append.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 5 + [vp, vp]
+    L.gqa_cache_append.restype = i32
+    L.gqa_cache_bytes.argtypes = [i64] * 6
+    L.gqa_cache_bytes.restype = ctypes.c_uint64
+    L.gqa_kv_head_for_query.argtypes = [i32] * 3
+    L.gqa_kv_head_for_query.restype = i32
+    L.gqa_window_start.argtypes = [i32, i32]
+    L.gqa_window_start.restype = i32
+    L.gqa_status_string.argtypes = [i32]
+    L.gqa_status_string.restype = ctypes.c_char_p
+    L.gqa_version.argtypes = []
+    L.gqa_version.restype = ctypes.c_char_p
+    return L
+
+
+def _status_string(s):
+    try:
+        return lib().gqa_status_string(int(s)).decode()
+    except Exception:  # pragma: no cover - only while reporting another error
+        return "?"
+
+
+def _check(status, what):
+    if status != 0:
+        raise GQAError(status, what)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float32:
+        return GQA_F32
+    if t.dtype == torch.bfloat16:
+        return GQA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t, name, dtype=None, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live in CUDA device memory")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _window(window):
+    return NO_WINDOW if window is None else int(window)
+
+
+def new_status(device):
+    """A zeroed device int32 status word."""
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def prefill(q, k, v, *, window=None, scale=None, seq_lens=None, out=None,
+            status=None, stream=None):
+    """o = GQA(q, k, v) over whole prompts.  q [B,Hq,T,d], k/v [B,Hkv,T,d]."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    st = status
+    _check(lib().gqa_prefill(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k, "k", q.dtype, dev), _ptr(v, "v", q.dtype, dev),
+        _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
+        B, Hq, Hkv, T, d, _window(window), float(scale),
+        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_prefill")
+    return out
+
+
+def decode_workspace_bytes(dtype, B, Hq, Hkv, C, d):
+    code = GQA_BF16 if dtype == torch.bfloat16 else GQA_F32
+    return int(lib().gqa_decode_workspace_bytes(code, B, Hq, Hkv, C, d))
+
+
+def decode_workspace(q, k_cache):
+    """A device workspace large enough for decode on these shapes."""
+    B, Hq, d = q.shape
+    Hkv, C = k_cache.shape[1], k_cache.shape[2]
+    n = decode_workspace_bytes(q.dtype, B, Hq, Hkv, C, d)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+
+
+def decode(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,
+           workspace=None, status=None, stream=None):
+    """One new token per sequence: q [B,Hq,d], caches [B,Hkv,C,d],
+    seq_lens [B] int32 counting the cached cells including the new token."""
+    B, Hq, d = q.shape
+    Hkv, C = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, C, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    if workspace is None:
+        workspace = decode_workspace(q, k_cache)
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_decode(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
+        _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
+        workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
+        "gqa_decode")
+    return out
+
+
+def cache_append(k_cache, v_cache, k_new, v_new, seq_lens, *, status=None, stream=None):
+    """Write k_new/v_new [B,Hkv,t_new,d] at cells [len_b, len_b+t_new) and
+    advance seq_lens in place (all-or-nothing on the device)."""
+    B, Hkv, C, d = k_cache.shape
+    t_new = k_new.shape[2]
+    if k_new.shape != (B, Hkv, t_new, d) or v_new.shape != k_new.shape:
+        raise ValueError("new K/V shape mismatch")
+    dev = k_cache.device
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_cache_append(
+        _dtype_code(k_cache), _ptr(k_cache, "k_cache"), _ptr(v_cache, "v_cache", k_cache.dtype, dev),
+        _ptr(k_new, "k_new", k_cache.dtype, dev), _ptr(v_new, "v_new", k_cache.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hkv, C, d, t_new,
+        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_cache_append")
+    return st
+
+
+def cache_bytes(L, B, T, Hkv, d, elem_bytes):
+    return int(lib().gqa_cache_bytes(L, B, T, Hkv, d, elem_bytes))
+
+
+def kv_head_for_query(h, Hq, Hkv):
+    g = lib().gqa_kv_head_for_query(h, Hq, Hkv)
+    return None if g < 0 else g
+
+
+def window_start(t, window):
+    s = lib().gqa_window_start(t, _window(window))
+    return None if s < 0 else s
+
+
+def version():
+    return lib().gqa_version().decode()

@@ -1,0 +1,176 @@
+/*
+ * gqa.h -- C ABI of the B200 (sm_100a) grouped-query attention library.
+ *
+ * Grouped-query attention (GQA): Hq query heads share Hkv key/value heads in
+ * groups of r = Hq/Hkv adjacent heads; query head h reads KV head
+ * g(h) = floor(h/r) in place (no repeat-interleave copy is made).  Each query
+ * row normalises softmax(scale * q.k) over its permitted key cells only and
+ * mixes the shared value rows.
+ *
+ * Sources (page title, section):
+ *   [P1] "Share key/value heads and make context explicit" (practical LLM in
+ *        Rust, ch. 18): "Give each query head an explicit shared KV head"
+ *        (head map, score, normalisation, value mix), "Intersect the window
+ *        with the context already permitted" (window w counts the current
+ *        cell and at most w-1 earlier cells; zero window refused; inactive
+ *        padded queries have zero output), "Extend the existing full and
+ *        cached attention paths" (decode reads the shared cache lane over
+ *        the eligible suffix; the cache refuses to exceed capacity and a
+ *        failed operation never partly advances it), "Count learned weights
+ *        and retained cache data separately" (physical cache [B,Hkv,C,d]).
+ *   [P3] "GQA, FlashAttention and the KV cache": "Computing the cache
+ *        requirement" (M_KV = 2 L B T Hkv d e), "The important mask bug with
+ *        a cache" (a single new token sees the whole cached past).
+ *   [P4] "How do you implement grouped query attention (GQA)?": Step 1
+ *        (shapes [B,H,T,d] and [B,G,T,d]), Step 2 (head map), the
+ *        implementation's tril(s - t) mask offset.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are contiguous row-major device buffers owned by the
+ *     caller.  The library allocates no device memory and keeps no state.
+ *   - Element type: GQA_F32 (float) or GQA_BF16 (bfloat16 storage, fp32
+ *     arithmetic).  All tensors of one call share the type.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  Host-detectable errors are returned
+ *     before anything is enqueued and leave every buffer untouched.
+ *   - `window` is GQA_NO_WINDOW (-1) for plain causal attention, else a
+ *     positive cell count that includes the current cell.  0 and values
+ *     below -1 return GQA_ERR_WINDOW.
+ *   - Device-resident lengths are validated on the device: an invalid
+ *     length sets *dev_status (int32, device memory) to a gqa_status code
+ *     (the first error wins; the library never clears it, so zero it before
+ *     the calls you want to check).  Outputs of a failed call hold zeros
+ *     and a failed append writes nothing.  No call traps.
+ */
+#ifndef GQA_H
+#define GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *gqa_stream_t; /* same type as cudaStream_t */
+
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype;
+
+typedef enum {
+  GQA_OK = 0,
+  GQA_ERR_NULL = 1,        /* a required pointer is NULL */
+  GQA_ERR_SHAPE = 2,       /* a size is negative, or Hq/Hkv/d is not positive */
+  GQA_ERR_GROUPS = 3,      /* Hq is not a multiple of Hkv */
+  GQA_ERR_WINDOW = 4,      /* window == 0 or window < -1 */
+  GQA_ERR_CAPACITY = 5,    /* a length is negative or exceeds T / C */
+  GQA_ERR_OVERFLOW = 6,    /* an element count overflows int64 / size_t */
+  GQA_ERR_UNSUPPORTED = 7, /* d, dtype or alignment outside the compiled kernels */
+  GQA_ERR_WORKSPACE = 8,   /* workspace NULL or smaller than required */
+  GQA_ERR_CUDA = 9,        /* a CUDA runtime call or launch failed */
+  GQA_ERR_DEVICE = 10,     /* the current device is not sm_100 */
+  GQA_ERR_TIMEOUT = 11     /* a kernel's bounded internal wait ran out (set
+                              in *dev_status only) */
+} gqa_status;
+
+#define GQA_NO_WINDOW (-1)
+
+/* Largest head width the kernels accept (fp32 and the generic bf16 path). */
+#define GQA_MAX_HEAD_DIM 256
+
+/*
+ * gqa_prefill -- full causal (optionally windowed) pass over a prompt.
+ * [P1] "Give each query head an explicit shared KV head" and "Intersect the
+ * window ...": for batch row b, query head h and active cell t < n_b, the
+ * permitted keys are j in [max(0, t-(w-1)), t] of KV head g(h); rows with
+ * t >= n_b are written as zeros.
+ *
+ *   q        [B,Hq,T,d]   queries (already position-rotated)
+ *   k, v     [B,Hkv,T,d]  keys (rotated) and values of the same cells
+ *   o        [B,Hq,T,d]   output; the head concatenation [B,T,Hq*d] of the
+ *                         pages is its transpose (the output projection W_o
+ *                         is not applied)
+ *   seq_lens device int32 [B] giving n_b in [0, T], or NULL for n_b = T
+ *   scale    score multiplier (1/sqrt(d) in the pages)
+ *   dev_status device int32, may be NULL when seq_lens is NULL
+ * bf16 with d in {64, 128} runs on the tcgen05 tensor cores; other d up to
+ * GQA_MAX_HEAD_DIM and fp32 run on CUDA cores with fp32 FMAs.
+ */
+gqa_status gqa_prefill(gqa_dtype dtype, const void *q, const void *k,
+                       const void *v, void *o, const int32_t *seq_lens,
+                       int B, int Hq, int Hkv, int T, int d, int window,
+                       float scale, int32_t *dev_status, gqa_stream_t stream);
+
+/*
+ * gqa_decode -- one new query token per sequence against the KV cache.
+ * [P1] "Extend the existing full and cached attention paths" and [P3] "The
+ * important mask bug with a cache": seq_lens[b] = n_b counts the cached
+ * cells INCLUDING the current token (append it first with
+ * gqa_cache_append); the query sits at cell n_b - 1 and reads cells
+ * [max(0, n_b - w), n_b) of its shared lane.  n_b = 0 gives a zero output.
+ *
+ *   q        [B,Hq,d]      the new token's queries
+ *   k_cache, v_cache [B,Hkv,C,d]  caches of capacity C
+ *   o        [B,Hq,d]      output
+ *   seq_lens device int32 [B], each in [0, C]
+ *   workspace / workspace_bytes  device scratch of at least
+ *            gqa_decode_workspace_bytes(...) bytes, 256-byte aligned; its
+ *            contents need no initialisation and are not preserved
+ *   dev_status device int32 (required)
+ * bf16 with d in {64, 128}: split-K flash-decode (bulk-copy fed shared
+ * memory ring, group heads stacked per CTA) plus a merge pass.
+ */
+gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
+                      const void *v_cache, void *o, const int32_t *seq_lens,
+                      int B, int Hq, int Hkv, int C, int d, int window,
+                      float scale, void *workspace, size_t workspace_bytes,
+                      int32_t *dev_status, gqa_stream_t stream);
+
+/* Workspace gqa_decode needs for these sizes (0 means none); 0 is also
+ * returned for invalid sizes, which gqa_decode then rejects. */
+size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,
+                                  int C, int d);
+
+/*
+ * gqa_cache_append -- write t_new new cells per sequence and advance the
+ * lengths.  [P1] "Count learned weights and retained cache data separately"
+ * and "Extend the existing full and cached attention paths": the cache
+ * keeps every row up to its fixed capacity (no eviction), refuses to exceed
+ * it, and never partly advances.
+ *
+ *   k_cache, v_cache [B,Hkv,C,d]  written at cells [len_b, len_b + t_new)
+ *   k_new, v_new     [B,Hkv,t_new,d]
+ *   seq_lens         device int32 [B], in/out: len_b += t_new on success
+ *   dev_status       device int32 (required)
+ * All-or-nothing: if any len_b < 0 or len_b + t_new > C, *dev_status is set
+ * to GQA_ERR_CAPACITY and neither the caches nor the lengths change.
+ */
+gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,
+                            const void *k_new, const void *v_new,
+                            int32_t *seq_lens, int B, int Hkv, int C, int d,
+                            int t_new, int32_t *dev_status,
+                            gqa_stream_t stream);
+
+/* [P3] "Computing the cache requirement": 2*L*B*T*Hkv*d*e bytes for L
+ * layers; 0 if any argument is negative or the product overflows uint64. */
+uint64_t gqa_cache_bytes(int64_t L, int64_t B, int64_t T, int64_t Hkv,
+                         int64_t d, int64_t elem_bytes);
+
+/* [P1] kv_head_for_query: g(h) = floor(h / (Hq/Hkv)); -1 when Hq or Hkv is
+ * not positive, Hq % Hkv != 0, or h is outside [0, Hq). */
+int gqa_kv_head_for_query(int h, int Hq, int Hkv);
+
+/* [P1] causal_window_start with segment start 0: the first permitted key
+ * cell of query cell t, max(0, t - (w-1)) (0 for GQA_NO_WINDOW); -1 for an
+ * invalid window or t < 0. */
+int gqa_window_start(int t, int window);
+
+/* Static English text for a status code (never NULL). */
+const char *gqa_status_string(gqa_status status);
+
+/* Library version, e.g. "0.1.0". */
+const char *gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GQA_H */
