@@ -33,7 +33,7 @@ def _cuda(*ts):
 def test_prefill_worked_example(cuda_lib, dtype):
     g = oracle_pins.golden("worked_example.json")
     q, k, v = oracle_pins.worked_example_inputs()
-    qt, kt, vt = _cuda(*(torch.from_numpy(x).to(dtype) for x in (q, k, v)))
+    qt, kt, vt = _cuda(*(torch.from_numpy(np.ascontiguousarray(x)).to(dtype) for x in (q, k, v)))
     for case in g["cases"]:
         o = cuda_lib.prefill(qt, kt, vt, window=case["window"])
         merged = f64(o)[0, :, -1, :].reshape(-1).tolist()
