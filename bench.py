@@ -1,0 +1,419 @@
+"""Benchmark of the GQA hot path on B200 (one JSON line on rank 0).
+
+A step is one pass of the decode hot path over one batch: reset the lengths
+to the cached count, append the new token's K/V to the cache
+(gqa_cache_append), then decode it against the cache (gqa_decode: head map,
+permitted window, scores, online softmax, value mix, split-K merge).
+The default workload is bf16 decode with B=8, Hq=32, Hkv=8, d=128 and 8000
+cached cells per sequence (8001 keys read with the new token).
+
+value  = algorithmic bytes per step x steps x ranks / max-over-ranks time,
+         algorithmic bytes = K+V of every permitted cell + Q + O + the
+         appended rows (read and written)
+e2e    = the same through the public API with host buffers: pinned host->
+         device copies of q and the new K/V, and the device->host read of o,
+         inside the timed region
+roofline = the split-K decode (split + merge kernels) against the measured
+         HBM copy bandwidth
+cpu_baseline = the fp64 oracle on this host's cores on a bounded sample
+
+Usage: python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                       [--workload NAME]
+Multi-GPU (torchrun): every rank runs its own independent batch (replicas,
+weak scaling; the path has no exchange step), timing is max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from grouped_query_attention_03_b200 import synthetic, workloads  # noqa: E402
+
+METRIC = "decode KV-cache HBM GB/s (% of 8 TB/s); prefill TFLOP/s (% bf16 peak)"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": 1590.0}, "fallback"
+
+
+class ClockSampler:
+    """SM clocks and clock-event (throttle) reasons sampled every ~1 ms by NVML
+    on a background thread while the timed region runs."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown",
+               0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap", 0x80: "hw_power_brake"}
+
+    def __init__(self, gpu_index, period_s=0.001):
+        self.gpu = gpu_index
+        self.period = period_s
+        self.sm, self.smax, self.mask = [], None, 0
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            self.ok = True
+        except Exception:  # no NVML: report no samples rather than guess
+            return self
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+        return self
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                self.sm.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.mask |= int(self.get_reasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self.stop.set()
+            self.thread.join(timeout=2)
+        return False
+
+    def summary(self):
+        reasons = sorted(n for bit, n in self.REASONS.items() if self.mask & bit)
+        return {"sm_mhz": statistics.median(self.sm) if self.sm else None,
+                "sm_max_mhz": self.smax, "reasons": reasons, "samples": len(self.sm),
+                "source": "nvml" if self.ok else "unavailable"}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def dist_max(x, device):
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.barrier()
+
+
+# --------------------------------------------------------------- workloads
+def decode_shape(w, window):
+    """(window, cached cells per sequence, capacity) of a decode step.  The
+    sliding-window workload decodes after its whole prompt is cached."""
+    if window is None and w.decode_steps and w.windows[0] is not None:
+        window = w.windows[0]
+    if w.ragged:
+        cached = synthetic.lengths_uniform(w.B, w.ragged[0], w.ragged[1], w.seed).tolist()
+        return window, cached, w.ragged[1] + 1
+    n = w.cached or w.T
+    return window, [n] * w.B, n + 1
+
+
+class DecodeStep:
+    """Append one token per sequence and decode it; the lengths are reset to
+    the cached count first so every step reads the same number of cells."""
+
+    def __init__(self, w, device, Hkv=None, window=None):
+        from grouped_query_attention_03_b200 import gqa
+        self.gqa = gqa
+        self.w = w
+        self.Hkv = Hkv or w.Hkv
+        self.window, self.cached, self.C = decode_shape(w, window)
+        B, Hq, d = w.B, w.Hq, w.d
+        C = self.C
+        self.q, self.kc, self.vc = [t.to(device) for t in synthetic.decode_inputs(
+            B, Hq, self.Hkv, C, d, w.seed, std=w.std)]
+        self.kn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=21).to(device)
+        self.vn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=22).to(device)
+        self.lens0 = torch.tensor(self.cached, dtype=torch.int32, device=device)
+        self.lens = self.lens0.clone()
+        self.o = torch.empty_like(self.q)
+        self.ws = gqa.decode_workspace(self.q, self.kc)
+        self.status = gqa.new_status(device)
+        n = np.array(self.cached) + 1
+        eff = np.minimum(n, window) if window else n
+        e = 2  # bf16
+        self.kv_bytes = int(2 * self.Hkv * eff.sum() * d * e)
+        self.qo_bytes = int(2 * B * Hq * d * e)
+        self.append_bytes = int(2 * 2 * B * self.Hkv * d * e)
+        self.decode_bytes = self.kv_bytes + self.qo_bytes
+        self.step_bytes = self.decode_bytes + self.append_bytes
+        self.launches_per_step = 4  # append copy + commit, split + merge
+
+    def run(self, ev=None):
+        self.lens.copy_(self.lens0, non_blocking=True)
+        self.gqa.cache_append(self.kc, self.vc, self.kn, self.vn, self.lens, status=self.status)
+        if ev is not None:
+            ev[0].record()
+        self.gqa.decode(self.q, self.kc, self.vc, self.lens, window=self.window, out=self.o,
+                        workspace=self.ws, status=self.status)
+        if ev is not None:
+            ev[1].record()
+
+    def run_host(self, hq, hkn, hvn, ho):
+        """One step through the public API from pinned host buffers."""
+        self.q.copy_(hq, non_blocking=True)
+        self.kn.copy_(hkn, non_blocking=True)
+        self.vn.copy_(hvn, non_blocking=True)
+        self.run()
+        ho.copy_(self.o, non_blocking=True)
+
+    def describe(self):
+        w = self.w
+        d = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": self.Hkv, "d": w.d,
+             "window": self.window, "capacity": self.C,
+             "keys_read_per_seq": "cached+1 (the appended token)",
+             "l2": "inputs exceed the 126 MB L2; no flush" if self.kv_bytes > 126e6
+             else "L2 flushed between steps (256 MB write)"}
+        if w.ragged:
+            d["cached_lengths"] = f"uniform [{w.ragged[0]}, {w.ragged[1]}], seed {w.seed}"
+        else:
+            d["cached"] = w.cached
+        return d
+
+
+def oracle_decode_sample(step, max_seconds):
+    """Time the fp64 oracle on a bounded sample of the same decode step."""
+    import oracle
+    cores = oracle.set_threads(0)
+    B = step.w.B
+    nb = B
+    q = step.q.float().cpu().double().numpy()
+    kc = step.kc.float().cpu().double().numpy()
+    vc = step.vc.float().cpu().double().numpy()
+    lens = np.array(step.cached) + 1
+    # one calibration call on a single sequence, then size the sample
+    t0 = time.perf_counter()
+    oracle.decode(q[:1], kc[:1], vc[:1], lens[:1], window=step.window)
+    per_seq = max(time.perf_counter() - t0, 1e-4)
+    nb = int(max(1, min(B, max_seconds / per_seq)))
+    reps = max(1, int(max_seconds / (per_seq * nb)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.decode(q[:nb], kc[:nb], vc[:nb], lens[:nb], window=step.window)
+    dt = time.perf_counter() - t0
+    n = lens[:nb]
+    eff = np.minimum(n, step.window) if step.window else n
+    bytes_ = reps * (2 * step.Hkv * eff.sum() * step.w.d * 2 + 2 * nb * step.w.Hq * step.w.d * 2)
+    return {"value": bytes_ / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x decode of {nb}/{B} sequences (fp64, all permitted cells)",
+            "seconds": dt}
+
+
+def flush_l2(buf):
+    buf.zero_()
+
+
+def run_gpu(args, world, rank, local):
+    from grouped_query_attention_03_b200 import build as gbuild
+    gbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = workloads.BY_NAME[args.workload]
+    step = DecodeStep(w, device, Hkv=args.hkv, window=args.window)
+    stream = torch.cuda.current_stream(device)
+    need_flush = step.kv_bytes <= 126e6
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=device) if need_flush else None
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush_l2(flush)
+        step.run()
+    torch.cuda.synchronize(device)
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} after warm-up")
+
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(local) as clocks:
+        if flush is None:
+            start.record(stream)
+            for i in range(K):
+                step.run(dec_ev[i])
+            end.record(stream)
+            torch.cuda.synchronize(device)
+            total_ms = start.elapsed_time(end)
+        else:
+            # flush between steps; time only the steps (events around each)
+            step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(K)]
+            for i in range(K):
+                flush_l2(flush)
+                step_ev[i][0].record(stream)
+                step.run(dec_ev[i])
+                step_ev[i][1].record(stream)
+            torch.cuda.synchronize(device)
+            total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    barrier()
+    total_ms = dist_max(total_ms, device)
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+    dec_avg_ms = statistics.mean(dec_ms)
+
+    # end to end through the public API with pinned host buffers
+    hq = step.q.cpu().pin_memory()
+    hkn = step.kn.cpu().pin_memory()
+    hvn = step.vn.cpu().pin_memory()
+    ho = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    for _ in range(2):
+        step.run_host(hq, hkn, hvn, ho)
+    torch.cuda.synchronize(device)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for i in range(K):
+        if flush is not None:
+            flush_l2(flush)
+        e0.record(stream)
+        step.run_host(hq, hkn, hvn, ho)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms += e0.elapsed_time(e1)
+    e2e_ms = dist_max(e2e_ms, device)
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} after timing")
+
+    peaks, peak_kind = measured_peaks()
+    value = step.step_bytes * K * world / (total_ms / 1e3) / 1e9
+    achieved = step.decode_bytes / (dec_avg_ms / 1e3) / 1e9
+    h2d = hq.numel() * hq.element_size() + hkn.numel() * hkn.element_size() * 2
+    d2h = ho.numel() * ho.element_size()
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = oracle_decode_sample(step, args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) rounded to bf16)",
+            "config": dict(step.describe(), parallelism=f"replicas x{world}"),
+            "frac_of_spec_8TBs": round(value / SPEC_HBM_GBS, 4),
+            "roofline": {"bound": "hbm", "kernel": "gqa_decode (split_kernel + merge_kernel)",
+                         "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
+                         "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4),
+                         "frac_of_spec_8TBs": round(achieved / SPEC_HBM_GBS, 4),
+                         "bytes_per_launch": step.decode_bytes,
+                         "avg_launch_us": round(dec_avg_ms * 1e3, 3),
+                         "traffic": args.traffic},
+            "e2e": {"value": round(step.step_bytes * K * world / (e2e_ms / 1e3) / 1e9, 2),
+                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": step.launches_per_step * K,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+        }
+    return line
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: fp64 on the host cores, bounded."""
+    if rank != 0:
+        return None
+    w = workloads.BY_NAME[args.workload]
+    step = DecodeStep.__new__(DecodeStep)
+    step.w = w
+    step.Hkv = args.hkv or w.Hkv
+    step.window, step.cached, step.C = decode_shape(w, args.window)
+    B, Hq, d = w.B, w.Hq, w.d
+    C = step.C
+    step.q, step.kc, step.vc = synthetic.decode_inputs(B, Hq, step.Hkv, C, d, w.seed, std=w.std)
+    budget = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_decode_sample(step, budget)
+    samples = [oracle_decode_sample(step, budget) for _ in range(args.steps)]
+    secs = sum(s["seconds"] for s in samples)
+    value = statistics.mean(s["value"] for s in samples)
+    n = np.array(step.cached) + 1
+    desc = {"workload": w.name, "B": B, "Hq": Hq, "Hkv": step.Hkv, "d": d, "window": step.window,
+            "capacity": C, "parallelism": "oracle on host cores"}
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / max(1, args.steps) * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": desc,
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "kind": "oracle",
+                         "cores": samples[0]["cores"], "sample": samples[0]["sample"]},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["own", "reference"], default="own")
+    ap.add_argument("--workload", default=workloads.DECODE_B8_N8000.name)
+    ap.add_argument("--hkv", type=int, default=None, help="override Hkv (ragged MQA/MHA endpoints)")
+    ap.add_argument("--window", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per launch for the roofline (null if unknown)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        # The oracle runs on rank 0 only; the other ranks exit without work.
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        line = run_gpu(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
