@@ -168,7 +168,7 @@ class DecodeStep:
         self.ws = gqa.decode_workspace(self.q, self.kc)
         self.status = gqa.new_status(device)
         n = np.array(self.cached) + 1
-        eff = np.minimum(n, window) if window else n
+        eff = np.minimum(n, self.window) if self.window else n
         e = 2  # bf16
         self.kv_bytes = int(2 * self.Hkv * eff.sum() * d * e)
         self.qo_bytes = int(2 * B * Hq * d * e)

@@ -296,3 +296,30 @@ def test_swa_t32768_decode_steps(cuda_lib):
         want = oracle.decode(f64(qn), k64, v64, [n], window=w.windows[0])
         worst = max(worst, assert_close(o, want, torch.bfloat16, f"step {step}")[0])
     assert int(st.item()) == 0 and lens.tolist() == [C]
+
+
+def test_prefill_swa_t32768_sampled_rows(cuda_lib):
+    """Sliding-window prefill at full size (B=1, Hq=32, Hkv=8, d=128,
+    T=32768, w=4096), checked on a stratified sample the oracle computes row
+    by row: every row t < 4096 of heads 0 and 31 (the window's ramp), and all
+    32 heads at 64 seeded random cells."""
+    w = workloads.SWA_T32768
+    window = w.windows[0]
+    q, k, v = synthetic.qkv_prefill(w.B, w.Hq, w.Hkv, w.T, w.d, w.seed, std=w.std)
+    o = cuda_lib.prefill(*_cuda(q, k, v), window=window)
+    torch.cuda.synchronize()
+    r = w.Hq // w.Hkv
+    for h in (0, w.Hq - 1):
+        g = h // r
+        T0 = window
+        want = oracle.prefill(f64(q[:, h:h + 1, :T0]), f64(k[:, g:g + 1, :T0]),
+                              f64(v[:, g:g + 1, :T0]), window=window)
+        assert_close(o[:, h:h + 1, :T0], want, torch.bfloat16, f"ramp rows head {h}")
+    k64, v64 = f64(k), f64(v)
+    rng = np.random.default_rng(w.seed)
+    cells = sorted(rng.choice(np.arange(window, w.T), size=64, replace=False).tolist())
+    got, want = [], []
+    for t in cells:
+        want.append(oracle.decode(f64(q[:, :, t]), k64, v64, [t + 1], window=window))
+        got.append(f64(o[:, :, t]))
+    assert_close(np.stack(got), np.stack(want), torch.bfloat16, "random rows")
