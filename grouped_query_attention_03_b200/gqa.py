@@ -27,8 +27,11 @@ STATUS_NAMES = {
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_prefill", "gqa_decode", "gqa_decode_workspace_bytes",
-           "gqa_cache_append", "gqa_cache_bytes", "gqa_kv_head_for_query",
-           "gqa_window_start", "gqa_status_string", "gqa_version")
+           "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
+           "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
+           "gqa_version")
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # GQA_NOALLOC_SCRATCH_BYTES in include/gqa.h
 
 
 class GQAError(RuntimeError):
@@ -60,6 +63,8 @@ def _declare(L):
     L.gqa_prefill.restype = i32
     L.gqa_decode.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, sz, vp, vp]
     L.gqa_decode.restype = i32
+    L.gqa_decode_noalloc.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, vp]
+    L.gqa_decode_noalloc.restype = i32
     L.gqa_decode_workspace_bytes.argtypes = [i32] * 6
     L.gqa_decode_workspace_bytes.restype = sz
     L.gqa_cache_append.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 5 + [vp, vp]
@@ -184,6 +189,30 @@ def decode(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,
         _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
         workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
         "gqa_decode")
+    return out
+
+
+def decode_noalloc(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,
+                   status=None, stream=None):
+    """decode() without a workspace argument, for callers that cannot
+    allocate device memory: the library's fixed device array serves as the
+    workspace (see gqa_decode_noalloc in include/gqa.h)."""
+    B, Hq, d = q.shape
+    Hkv, C = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, C, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_decode_noalloc(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
+        _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
+        _stream(stream, dev)), "gqa_decode_noalloc")
     return out
 
 

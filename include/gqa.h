@@ -130,6 +130,40 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
 size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,
                                   int C, int d);
 
+/* Size of the fixed device array gqa_decode_noalloc uses as its workspace. */
+#define GQA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * gqa_decode_noalloc -- gqa_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart; this is a library convenience.
+ *
+ * Some callers cannot call cudaMalloc: a host application that passes this
+ * library pointers from its own fixed memory pool and forbids any other
+ * allocation, a latency-critical loop that cannot accept cudaMalloc's
+ * implicit device synchronisation, or a foreign-language caller that only
+ * receives device pointers.  This entry point takes the same arguments as
+ * gqa_decode minus the workspace and runs the same kernels, using as
+ * workspace a fixed GQA_NOALLOC_SCRATCH_BYTES array in device memory that
+ * the library defines (every GPU that loads the library holds it until the
+ * process exits).  It allocates nothing.
+ *
+ *   - Sizes whose workspace (gqa_decode_workspace_bytes) exceeds
+ *     GQA_NOALLOC_SCRATCH_BYTES return GQA_ERR_WORKSPACE; nothing is
+ *     enqueued.  All other arguments and errors are those of gqa_decode.
+ *   - All calls on a device share the one array, which keeps the last
+ *     call's contents; nothing in it needs to start at zero.  Calls whose
+ *     kernels may overlap on the GPU (unordered streams) race on it: order
+ *     them on one stream or with events.
+ *   - The first call on each device looks up the array's address (with that
+ *     device current) and caches it; make that first call before any stream
+ *     capture begins.  A failed lookup returns GQA_ERR_CUDA.
+ */
+gqa_status gqa_decode_noalloc(gqa_dtype dtype, const void *q,
+                              const void *k_cache, const void *v_cache,
+                              void *o, const int32_t *seq_lens, int B, int Hq,
+                              int Hkv, int C, int d, int window, float scale,
+                              int32_t *dev_status, gqa_stream_t stream);
+
 /*
  * gqa_cache_append -- write t_new new cells per sequence and advance the
  * lengths.  [P1] "Count learned weights and retained cache data separately"
