@@ -209,6 +209,58 @@ class DecodeStep:
         return d
 
 
+class PrefillStep:
+    """One gqa_prefill over a whole prompt batch."""
+
+    def __init__(self, w, device, window):
+        from grouped_query_attention_03_b200 import gqa
+        self.gqa, self.w, self.window = gqa, w, window
+        self.q, self.k, self.v = [t.to(device) for t in synthetic.qkv_prefill(
+            w.B, w.Hq, w.Hkv, w.T, w.d, w.seed, std=w.std)]
+        self.o = torch.empty_like(self.q)
+        t = np.arange(w.T)
+        lo = np.maximum(0, t - (window - 1)) if window else np.zeros_like(t)
+        self.pairs = int((t - lo + 1).sum())          # permitted pairs per (b, h)
+        self.flops = 4 * w.d * self.pairs * w.B * w.Hq  # QK^T + PV, 2 flops per MAC
+        self.in_bytes = sum(x.numel() * x.element_size() for x in (self.q, self.k, self.v))
+
+    def run(self):
+        self.gqa.prefill(self.q, self.k, self.v, window=self.window, out=self.o)
+
+    def describe(self):
+        w = self.w
+        return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
+                "window": self.window, "permitted_pairs_per_head": self.pairs}
+
+
+def measure_prefill(w, window, device, reps, warmup):
+    """Per-launch prefill time (CUDA events), L2 flushed between launches
+    when the inputs fit in L2."""
+    step = PrefillStep(w, device, window)
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=device) \
+        if step.in_bytes <= 126e6 else None
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize(device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for a, b in evs:
+        if flush is not None:
+            flush_l2(flush)
+        a.record()
+        step.run()
+        b.record()
+    torch.cuda.synchronize(device)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    peaks, kind = measured_peaks()
+    tflops = step.flops / (ms / 1e3) / 1e12
+    return step, {
+        **step.describe(), "tflops": round(tflops, 2), "ms": round(ms, 4),
+        "flops": step.flops, "frac_of_measured": round(tflops / peaks["bf16_tflops"], 4),
+        "peak_kind": f"{kind} bf16 matmul (burst)", "frac_of_spec_2250": round(tflops / 2250.0, 4),
+        "l2": "inputs exceed L2" if flush is None else "L2 flushed between launches"}
+
+
 def oracle_decode_sample(step, max_seconds):
     """Time the fp64 oracle on a bounded sample of the same decode step."""
     import oracle
@@ -312,6 +364,11 @@ def run_gpu(args, world, rank, local):
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after timing")
 
+    prefill_extra = None
+    if rank == 0 and not args.no_prefill:
+        prefill_extra = [measure_prefill(workloads.SWA_T32768, 4096, device, 10, 3)[1],
+                         measure_prefill(workloads.PREFILL_B4_T1024, None, device, 20, 3)[1],
+                         measure_prefill(workloads.PREFILL_B4_T1024, 256, device, 20, 3)[1]]
     peaks, peak_kind = measured_peaks()
     value = step.step_bytes * K * world / (total_ms / 1e3) / 1e9
     achieved = step.decode_bytes / (dec_avg_ms / 1e3) / 1e9
@@ -342,8 +399,42 @@ def run_gpu(args, world, rank, local):
             "gpu_launches": step.launches_per_step * K,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
+            "prefill": prefill_extra,
         }
     return line
+
+
+def run_gpu_prefill(args, world, rank, local):
+    """--phase prefill: the main line is prefill TFLOP/s on one workload."""
+    from grouped_query_attention_03_b200 import build as gbuild
+    gbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = workloads.BY_NAME[args.workload]
+    window = args.window if args.window is not None else w.windows[0]
+    barrier()
+    with ClockSampler(local) as clocks:
+        step, res = measure_prefill(w, window, device, args.steps, args.warmup)
+    ms = dist_max(res["ms"], device)
+    peaks, kind = measured_peaks()
+    value = step.flops * world / (ms / 1e3) / 1e12
+    if rank != 0:
+        return None
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal rounded to bf16)",
+        "config": dict(step.describe(), parallelism=f"replicas x{world}", l2=res["l2"]),
+        "roofline": {"bound": "tensor", "kernel": "pf::prefill_kernel",
+                     "achieved": res["tflops"], "peak": peaks["bf16_tflops"],
+                     "peak_kind": f"{kind} bf16 matmul (burst)", "unit": "TFLOP/s",
+                     "frac": res["frac_of_measured"], "frac_of_spec_2250": res["frac_of_spec_2250"],
+                     "flops_per_launch": step.flops, "avg_launch_us": round(res["ms"] * 1e3, 2),
+                     "traffic": args.traffic},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
 
 
 def run_reference(args, world, rank):
@@ -391,6 +482,9 @@ def main(argv=None):
     ap.add_argument("--window", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--phase", choices=["decode", "prefill"], default="decode")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill figures on the decode line")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch for the roofline (null if unknown)")
     args = ap.parse_args(argv)
@@ -406,7 +500,10 @@ def main(argv=None):
         return
     world, rank, local = dist_setup(args)
     try:
-        line = run_gpu(args, world, rank, local)
+        if args.phase == "prefill":
+            line = run_gpu_prefill(args, world, rank, local)
+        else:
+            line = run_gpu(args, world, rank, local)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
     finally:
