@@ -15,46 +15,73 @@
 // lane + c (an injective map: along the staircase of (c, lane) pairs each
 // step raises c, lane or both).
 //
-// Inside a CTA: warp 4 is the producer.  It walks the CTA's row range and
-// streams stages of up to ROWS rows of K and V (plus the group's r query rows
-// at the start of each lane segment) into a STAGES-deep shared-memory ring
-// with non-multicast bulk copies completing on mbarriers.  Warps 0-3 consume
-// each stage: warp w takes rows [w*RW, (w+1)*RW); within a warp LPR lanes
-// share one row, each lane holding E features (16-byte shared loads), and
-// the r query heads of the group are stacked so one K/V read serves all of
-// them.  Dot products use packed fp32x2 FMAs, are reduced across the row's
-// lanes by a transposed (reduce-scatter) shuffle tree, and the online
-// softmax max/sum run on warp shuffles.  At the end of a lane segment the
-// four warps' states are combined through shared memory into one partial.
-// A second kernel merges the partials of each lane and writes bf16 output.
+// Inside a CTA the last warp is the producer.  It walks the CTA's row range
+// and fills a STAGES-deep shared-memory ring: ROWS cache rows of K and of V
+// per stage, fetched by TMA tensor copies (no multicast) in 128-byte
+// swizzled 64-column boxes, plus the group's query rows (bulk copy) at the
+// start of each lane segment.  Each of the NWC compute warps owns 16 rows of
+// a stage.  The group's R <= 16 query heads are stacked as the rows of one
+// 16-row tile, so the scores of 16 cache rows are one 16x16 tile
+// S = Q K^T and the value mix one 16 x d tile O += P V, both on the tensor
+// cores (mma.sync m16n8k16, bf16 in, fp32 accumulate; the K and V operands
+// come straight from the swizzled stage with ldmatrix).  The online softmax
+// works on the accumulator fragments: row max and sum over the four lanes
+// that share a head row with warp shuffles, accumulators rescaled lazily
+// (only when a running max grows by more than 2^8).  Per cache row that is
+// about two tensor instructions and a handful of others, which keeps the SM
+// ahead of HBM even when 8 or 16 query heads share each K/V row; the
+// CUDA-core formulation cannot do that beyond one or two heads per row.
+// At the end of a lane segment the warps' states are combined through the
+// just-consumed stage buffer.  A lane covered by one CTA is written out
+// directly; otherwise the combined (m, l, acc) goes to the workspace and the
+// last CTA to finish that lane (a per-lane atomic counter, zeroed at the
+// start of every call) merges the lane's partials and writes bf16 output.
+// No CTA ever waits for another.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace gqa {
 namespace dec {
 
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
-constexpr int kComputeWarps = 4;
-constexpr int kThreads = (kComputeWarps + 1) * 32;
+constexpr float kLazyRescale = 8.0f;  // log2 units
+constexpr int kBR = 16;               // rows per compute warp per stage
+
+// Compute warps per CTA, CTAs per SM and ring depth (overridable when
+// building, for tuning).
+#ifndef GQA_DEC_NWC
+#define GQA_DEC_NWC 8
+#endif
+#ifndef GQA_DEC_MIN_BLOCKS
+#define GQA_DEC_MIN_BLOCKS 1
+#endif
+#ifndef GQA_DEC_STAGES
+#define GQA_DEC_STAGES 3
+#endif
 
 template <int D, int R>
 struct Cfg {
-  static constexpr int E = (D == 128 && R <= 4) ? 16 : 8;  // features / lane
-  static constexpr int LPR = D / E;                        // lanes per row
-  static constexpr int RPP = 32 / LPR;                     // rows per pass
-  static constexpr int NC = E / 8;                         // 16-B chunks / lane
-  static constexpr int ROWS = (D == 128) ? 64 : 128;       // rows per stage
-  static constexpr int RW = ROWS / kComputeWarps;          // rows per warp
-  static constexpr int NP = RW / RPP;                      // passes per stage
-  static constexpr int STAGES = 3;
-  static constexpr int KV_BYTES = ROWS * D * 2;
-  static constexpr int Q_BYTES = R * D * 2;
-  static constexpr int STAGE_BYTES = 2 * KV_BYTES + Q_BYTES;
-  static_assert(LPR >= R, "reduce-scatter needs at least R lanes per row");
-  static_assert(RW % RPP == 0, "whole passes per warp");
-  static_assert(kComputeWarps * R * (D + 2) * 4 <= 2 * KV_BYTES,
+  static constexpr int NWC = GQA_DEC_NWC;              // compute warps
+  static constexpr int MIN_BLOCKS = GQA_DEC_MIN_BLOCKS;  // CTAs per SM
+  static constexpr int THREADS = (NWC + 1) * 32;
+  static constexpr int ROWS = NWC * kBR;               // rows per stage
+  static constexpr int KB = D / 64;                    // 64-column boxes
+  static constexpr int BOX = ROWS * 128;               // bytes of one box
+  static constexpr int KV_BYTES = KB * BOX;            // K (or V) per stage
+  static constexpr int QRAW = ((R * D * 2 + 1023) / 1024) * 1024;
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES + QRAW;
+  static constexpr int STAGES = GQA_DEC_STAGES;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+  static constexpr int KS = D / 16;                    // k-steps of 16 features
+  static constexpr int NT = D / 8;                     // 8-feature output tiles
+  static_assert(R <= 16, "one 16-row tile holds the stacked heads");
+  static_assert(NWC * (2 * 16 + R * D) * 4 <= STAGE_BYTES,
                 "combine scratch must fit in one stage");
+  static_assert(STAGE_BYTES % 1024 == 0 && BOX % 1024 == 0, "swizzle alignment");
 };
 
 struct StageHdr {
@@ -63,18 +90,13 @@ struct StageHdr {
   int nrows;
   int flags;
   int slot;   // partial slot (lane + CTA index)
-  int pad[3];
-};
-
-struct WsHdr {
-  long long total;
-  long long per;
-  int valid;
-  int pad[11];
+  int c0;     // first CTA whose range touches the lane
+  int np;     // number of CTAs whose ranges touch the lane
+  int pad;
 };
 
 struct Params {
-  const __nv_bfloat16 *q, *kc, *vc;
+  const __nv_bfloat16 *q;
   __nv_bfloat16 *o;
   const int32_t *seq_lens;
   int B, Hq, Hkv, C, window;
@@ -83,8 +105,7 @@ struct Params {
   int nsub;   // sub-groups of at most R heads per KV head
   int VL;     // virtual lanes per batch row = Hkv * nsub
   int min_rows;
-  WsHdr *hdr;
-  long long *lane_start;  // [B*VL]
+  int *counters;          // [B*VL], zero at kernel start
   float2 *ml;             // [(grid + B*VL) * R]: (m, l)
   float *acc;             // [(grid + B*VL) * R * D]
   int32_t *status;
@@ -94,10 +115,18 @@ __device__ __forceinline__ int eligible(int n, int window) {
   return window > 0 ? min(n, window) : n;
 }
 
+// Byte offset of 16-byte chunk `ch` (0..7) of row `r` inside a 128-byte
+// swizzled box (the TMA swizzle XORs the chunk index with r mod 8).
+__device__ __forceinline__ int swz(int r, int ch) {
+  return r * 128 + ((ch ^ (r & 7)) << 4);
+}
+
 // -------------------------------------------------------------- producer
 template <int D, int R>
-__device__ void producer(const Params &p, unsigned char *smem, StageHdr *hdrs,
-                         uint64_t *full, uint64_t *empty) {
+__device__ void producer(const Params &p, const CUtensorMap *tmK,
+                         const CUtensorMap *tmV, unsigned char *smem,
+                         StageHdr *hdrs, uint64_t *full, uint64_t *empty,
+                         bool bad) {
   using K = Cfg<D, R>;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -116,28 +145,20 @@ __device__ void producer(const Params &p, unsigned char *smem, StageHdr *hdrs,
     }
     return true;
   };
-
-  // Pass 1: validity and the total eligible row count.
-  bool bad = false;
-  long long tot = 0;
-  for (int b = lane; b < p.B; b += 32) {
-    const int n = p.seq_lens[b];
-    bad |= (n < 0 || n > p.C);
-    tot += eligible(n, p.window);
+  if (lane == 0) {
+    tc::prefetch_tmap(tmK);
+    tc::prefetch_tmap(tmV);
   }
-  bad = __any_sync(0xffffffffu, bad);
+
+  // Pass 1: the total eligible row count (lengths already validated).
+  long long tot = 0;
+  for (int b = lane; b < p.B && !bad; b += 32) tot += eligible(p.seq_lens[b], p.window);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1)
     tot += __shfl_xor_sync(0xffffffffu, tot, off);
   const long long total = tot * p.VL;
   long long per = (total + G - 1) / G;
   if (per < p.min_rows) per = p.min_rows;
-  if (c == 0 && lane == 0) {
-    p.hdr->valid = bad ? 0 : 1;
-    p.hdr->total = total;
-    p.hdr->per = per;
-    if (bad) record_status(p.status, GQA_ERR_CAPACITY);
-  }
   const long long start = (long long)c * per;
   const long long end = min(total, start + per);
 
@@ -176,7 +197,6 @@ __device__ void producer(const Params &p, unsigned char *smem, StageHdr *hdrs,
     while (pos < end) {
       const int L = b * p.VL + vl;
       const long long SL = cum_b + (long long)vl * len;
-      if (row == 0 && seg_first && lane == 0) p.lane_start[L] = SL;
       const int nrows = (int)min((long long)min(K::ROWS, len - row), end - pos);
       const bool last = (row + nrows == len) || (pos + nrows == end);
       int st;
@@ -188,19 +208,24 @@ __device__ void producer(const Params &p, unsigned char *smem, StageHdr *hdrs,
         h.nrows = nrows;
         h.flags = (seg_first ? kFirst : 0) | (last ? kLast : 0);
         h.slot = L + c;
+        h.c0 = (int)(SL / per);
+        h.np = (int)((SL + len - 1) / per) - h.c0 + 1;
         const int g = vl / p.nsub, sub = vl % p.nsub;
         const int h0 = g * p.r + sub * R;
         const int rc = min(R, p.r - sub * R);
-        const uint32_t kvb = (uint32_t)nrows * D * 2;
         const uint32_t qb = seg_first ? (uint32_t)rc * D * 2 : 0u;
         unsigned char *base = smem + (size_t)st * K::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[st], 2 * kvb + qb);
-        const size_t src = (((size_t)b * p.Hkv + g) * p.C + lo + row) * D;
-        bulk_g2s(base, p.kc + src, kvb, &full[st]);
-        bulk_g2s(base + K::KV_BYTES, p.vc + src, kvb, &full[st]);
+        mbar_arrive_expect_tx(&full[st], 2 * K::KV_BYTES + qb);
+        // Whole boxes are fetched; rows past the segment are never used.
+        const int y = (b * p.Hkv + g) * p.C + lo + row;
+#pragma unroll
+        for (int kb = 0; kb < K::KB; ++kb) {
+          tc::tma_load_2d(base + kb * K::BOX, tmK, kb * 64, y, &full[st]);
+          tc::tma_load_2d(base + K::KV_BYTES + kb * K::BOX, tmV, kb * 64, y, &full[st]);
+        }
         if (seg_first)
-          bulk_g2s(base + 2 * K::KV_BYTES, p.q + ((size_t)b * p.Hq + h0) * D,
-                   qb, &full[st]);
+          bulk_g2s(base + 2 * K::KV_BYTES, p.q + ((size_t)b * p.Hq + h0) * D, qb,
+                   &full[st]);
       }
       __syncwarp();
       fills[st]++;
@@ -240,7 +265,7 @@ __device__ void producer(const Params &p, unsigned char *smem, StageHdr *hdrs,
     __syncwarp();
     fills[st]++;
   }
-  // Never leave a bulk copy in flight into shared memory of an exiting CTA.
+  // Never leave a copy in flight into shared memory of an exiting CTA.
   bool f2 = false;
 #pragma unroll
   for (int s = 0; s < K::STAGES; ++s)
@@ -248,219 +273,285 @@ __device__ void producer(const Params &p, unsigned char *smem, StageHdr *hdrs,
   if ((failed || f2) && lane == 0) record_status(p.status, kStatusTimeout);
 }
 
+// Barrier among the compute warps (an mbarrier counting one arrival per
+// warp, so a wait can give up instead of hanging).
+__device__ __forceinline__ void csync(uint64_t *comb, int &count, bool *failed) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(comb);
+  mbar_wait(comb, count & 1, failed);
+  count++;
+}
+
+// The last CTA to finish lane L merges its np partials (slots L+c0 ..):
+// m = max m_i, l = sum e^{m_i - m} l_i, o = sum e^{m_i - m} acc_i / l.
+// Runs on the compute warps; `scratch` holds 2 * R * NWC floats.
+template <int D, int R>
+__device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
+                           __nv_bfloat16 *out, int rc, float *scratch,
+                           uint64_t *comb, int &comb_count, bool *failed) {
+  using K = Cfg<D, R>;
+  constexpr int NT = K::NWC * 32;
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const float2 *ml = p.ml + (size_t)(L + c0) * R;
+  float *red = scratch;            // [NWC][R]
+  float *msm = scratch + K::NWC * R;  // [R] max, then [R] denominators
+  float *lsm = msm + R;
+  const int h_t = t % R;  // NT is a multiple of R
+  float lm = -INFINITY;
+  for (int idx = t; idx < np * R; idx += NT) lm = fmaxf(lm, ml[idx].x);
+#pragma unroll
+  for (int off = 16; off >= R; off >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, off));
+  if (lane < R) red[w * R + lane] = lm;
+  csync(comb, comb_count, failed);
+  if (t < R) {
+    float m = red[t];
+#pragma unroll
+    for (int i = 1; i < K::NWC; ++i) m = fmaxf(m, red[i * R + t]);
+    msm[t] = m;
+  }
+  csync(comb, comb_count, failed);
+  const float mh = msm[h_t];
+  float ld = 0.f;
+  for (int idx = t; idx < np * R; idx += NT) {
+    const float2 v = ml[idx];
+    ld += v.x == -INFINITY ? 0.f : exp2f(v.x - mh) * v.y;
+  }
+#pragma unroll
+  for (int off = 16; off >= R; off >>= 1) ld += __shfl_xor_sync(0xffffffffu, ld, off);
+  if (lane < R) red[w * R + lane] = ld;
+  csync(comb, comb_count, failed);
+  if (t < R) {
+    float l = 0.f;
+#pragma unroll
+    for (int i = 0; i < K::NWC; ++i) l += red[i * R + t];
+    lsm[t] = l;
+  }
+  csync(comb, comb_count, failed);
+  // one float4 of output per thread and pass; loads of all partials issued
+  // back to back
+  const float4 *acc4 = reinterpret_cast<const float4 *>(p.acc + (size_t)(L + c0) * R * D);
+  for (int q4 = t; q4 < R * D / 4; q4 += NT) {
+    const int h = q4 / (D / 4);
+    const float m = msm[h];
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int c = 0; c < np; ++c) {
+      const float mc = ml[c * R + h].x;
+      const float e = mc == -INFINITY ? 0.f : exp2f(mc - m);
+      const float4 a = acc4[(size_t)c * (R * D / 4) + q4];
+      x.x += e * a.x;
+      x.y += e * a.y;
+      x.z += e * a.z;
+      x.w += e * a.w;
+    }
+    if (h < rc) {
+      const float inv = 1.f / lsm[h];
+      *reinterpret_cast<uint2 *>(out + q4 * 4) =
+          make_uint2(pack_bf16(x.x * inv, x.y * inv), pack_bf16(x.z * inv, x.w * inv));
+    }
+  }
+}
+
 // ------------------------------------------------------------- consumers
+// Fragment layout of mma.m16n8k16 (g = lane / 4, t = lane % 4):
+//   A regs 0..3: (row g, cols 2t..2t+1), (row g+8, same), (row g, cols
+//                8+2t..), (row g+8, cols 8+2t..)
+//   B regs 0..1: (rows 2t..2t+1, col g), (rows 8+2t.., col g)
+//   C regs 0..3: (row g, cols 2t, 2t+1), (row g+8, cols 2t, 2t+1)
+// Tile rows are query heads; S columns are cache rows; O columns features.
 template <int D, int R>
 __device__ void consumer(const Params &p, unsigned char *smem,
                          const StageHdr *hdrs, uint64_t *full, uint64_t *empty,
-                         uint64_t *comb) {
+                         uint64_t *comb, int &merge_flag) {
   using K = Cfg<D, R>;
-  constexpr int E = K::E, LPR = K::LPR, NC = K::NC, NP = K::NP;
+  constexpr int NWC = K::NWC, KS = K::KS, NT = K::NT;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int sub = lane % LPR;          // feature slot within the row
-  const int rip = lane / LPR;          // row within a pass
-  const int h_lane = sub / (LPR / R);  // head whose score this lane ends with
+  const int g = lane >> 2, t = lane & 3;
   bool failed = false;
 
-  float2 q2[R][E / 2];
-  float2 acc[R][E / 2];
-  float m_run = -INFINITY, l_run = 0.f;
+  uint32_t qa[KS][4];      // Q tile, A operand, per 16-feature k-step
+  float o[NT][4];          // O tile accumulators
+  float m_run[2], l_run[2];  // head rows g and g + 8
   int stage_count = 0, comb_count = 0;
 
   while (true) {
     const int st = stage_count % K::STAGES;
     const uint32_t par = (stage_count / K::STAGES) & 1;
-    if (!mbar_wait(&full[st], par, &failed)) break;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], par, &failed))) break;
     const StageHdr hd = hdrs[st];
     if (hd.flags & kEnd) break;
     unsigned char *base = smem + (size_t)st * K::STAGE_BYTES;
-    const __nv_bfloat16 *sK = reinterpret_cast<const __nv_bfloat16 *>(base);
-    const __nv_bfloat16 *sV =
-        reinterpret_cast<const __nv_bfloat16 *>(base + K::KV_BYTES);
+    const uint32_t sK = smem_u32(base);
+    const uint32_t sV = smem_u32(base + K::KV_BYTES);
 
     if (hd.flags & kFirst) {
+      // The group's query rows (bf16, [rc][D]) -> A fragments; rows past the
+      // group are zero.
       const __nv_bfloat16 *sQ =
           reinterpret_cast<const __nv_bfloat16 *>(base + 2 * K::KV_BYTES);
       const int vl = hd.lane % p.VL;
       const int rc = min(R, p.r - (vl % p.nsub) * R);
 #pragma unroll
-      for (int h = 0; h < R; ++h) {
-#pragma unroll
-        for (int i = 0; i < NC; ++i) {
-          uint4 u = make_uint4(0, 0, 0, 0);
-          if (h < rc)
-            u = *reinterpret_cast<const uint4 *>(sQ + h * D + 8 * (sub + LPR * i));
-          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            q2[h][i * 4 + j] = make_float2(bf16lo_to_f32(w4[j]) * p.scale_log2,
-                                           bf16hi_to_f32(w4[j]) * p.scale_log2);
-        }
-#pragma unroll
-        for (int e = 0; e < E / 2; ++e) acc[h][e] = make_float2(0.f, 0.f);
+      for (int ks = 0; ks < KS; ++ks) {
+        const int c0 = ks * 16 + 2 * t;
+        qa[ks][0] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0) : 0u;
+        qa[ks][1] = g + 8 < rc ? *reinterpret_cast<const uint32_t *>(sQ + (g + 8) * D + c0) : 0u;
+        qa[ks][2] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0 + 8) : 0u;
+        qa[ks][3] = g + 8 < rc ? *reinterpret_cast<const uint32_t *>(sQ + (g + 8) * D + c0 + 8) : 0u;
       }
-      m_run = -INFINITY;
-      l_run = 0.f;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      m_run[0] = m_run[1] = -INFINITY;
+      l_run[0] = l_run[1] = 0.f;
     }
 
-    // ---- scores for this warp's rows of the stage
-    float s[NP];
+    const int nv = hd.nrows - w * kBR;  // valid rows of this warp's 16
+    if (nv < kBR && nv > 0) {
+      // Rows past the segment hold other data (maybe non-finite): zero this
+      // warp's share of them in V so 0 * V stays 0.
+      for (int idx = lane; idx < (kBR - nv) * (D / 8); idx += 32) {
+        const int row = w * kBR + nv + idx / (D / 8), ch = idx % (D / 8);
+        *reinterpret_cast<uint4 *>(base + K::KV_BYTES + (ch >> 3) * K::BOX +
+                                   swz(row, ch & 7)) = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+
+    if (nv > 0) {
+      // ---- S = Q K^T for this warp's 16 cache rows (two 8-row tiles)
+      float s[2][4];
 #pragma unroll
-    for (int pp = 0; pp < NP; ++pp) {
-      const int rr = w * K::RW + pp * K::RPP + rip;
-      const bool valid = rr < hd.nrows;
-      float2 dot[R];
+      for (int nt = 0; nt < 2; ++nt) {
+        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+        const int krow = w * kBR + nt * 8 + (lane & 7);
 #pragma unroll
-      for (int h = 0; h < R; ++h) dot[h] = make_float2(0.f, 0.f);
-      if (valid) {
+        for (int kk = 0; kk < KS / 2; ++kk) {
+          const int ch = 4 * kk + (lane >> 3);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sK + (ch >> 3) * K::BOX + swz(krow, ch & 7), b0, b1, b2, b3);
+          mma_16816(s[nt], qa[2 * kk], b0, b1);
+          mma_16816(s[nt], qa[2 * kk + 1], b2, b3);
+        }
+      }
+      // ---- online softmax on the fragments (log2 domain)
+      float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < NC; ++i) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(
-              sK + rr * D + 8 * (sub + LPR * i));
-          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 kf = make_float2(bf16lo_to_f32(w4[j]), bf16hi_to_f32(w4[j]));
+        for (int e = 0; e < 4; ++e) {
+          const int col = nt * 8 + 2 * t + (e & 1);
+          const float v = col < nv ? s[nt][e] * p.scale_log2 : -INFINITY;
+          s[nt][e] = v;
+          mx[e >> 1] = fmaxf(mx[e >> 1], v);
+        }
 #pragma unroll
-            for (int h = 0; h < R; ++h) ffma2(dot[h], q2[h][i * 4 + j], kf);
+      for (int i = 0; i < 2; ++i) {
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+        if (mx[i] > m_run[i] + kLazyRescale) {
+          const float alpha = exp2f(m_run[i] - mx[i]);  // 0 when m_run = -inf
+          l_run[i] *= alpha;
+          m_run[i] = mx[i];
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            o[n][2 * i] *= alpha;
+            o[n][2 * i + 1] *= alpha;
           }
         }
       }
-      // Transposed reduction over the LPR lanes of the row: each halving
-      // step trades half the heads with the partner lane, so the lane ends
-      // with the full dot product of head h_lane.
-      float v[R];
+      uint32_t pa[4];
 #pragma unroll
-      for (int h = 0; h < R; ++h) v[h] = dot[h].x + dot[h].y;
+      for (int nt = 0; nt < 2; ++nt) {
+        float pv[4];
 #pragma unroll
-      for (int nv = R, off = LPR / 2; off >= 1; off >>= 1) {
-        if (nv > 1) {
-          const int half = nv / 2;
-          const bool upper = (lane & off) != 0;
-#pragma unroll
-          for (int i = 0; i < half; ++i) {
-            const float send = upper ? v[i] : v[i + half];
-            const float keep = upper ? v[i + half] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-          }
-          nv = half;
-        } else {
-          v[0] += __shfl_xor_sync(0xffffffffu, v[0], off);
+        for (int e = 0; e < 4; ++e) {
+          const float msub = m_run[e >> 1] == -INFINITY ? 0.f : m_run[e >> 1];
+          pv[e] = exp2f(s[nt][e] - msub);
         }
+        pa[2 * nt] = pack_bf16(pv[0], pv[1]);
+        pa[2 * nt + 1] = pack_bf16(pv[2], pv[3]);
+        // the denominator sums exactly the bf16 weights the MMA uses
+        l_run[0] += bf16lo_to_f32(pa[2 * nt]) + bf16hi_to_f32(pa[2 * nt]);
+        l_run[1] += bf16lo_to_f32(pa[2 * nt + 1]) + bf16hi_to_f32(pa[2 * nt + 1]);
       }
-      s[pp] = valid ? v[0] : -INFINITY;
-    }
-
-    // ---- online softmax (log2 domain; q carries scale*log2(e))
-    float mx = s[0];
+      // ---- O += P V (A = P over the 16 cache rows, B = V rows from smem)
+      const int vrow = w * kBR + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-    for (int pp = 1; pp < NP; ++pp) mx = fmaxf(mx, s[pp]);
-#pragma unroll
-    for (int off = LPR; off < 32; off <<= 1)
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const float m_new = fmaxf(m_run, mx);
-    const float msub = m_new == -INFINITY ? 0.f : m_new;
-    const float alpha = exp2f(m_run - msub);  // 0 when m_run = -inf
-    float lsum = 0.f;
-#pragma unroll
-    for (int pp = 0; pp < NP; ++pp) {
-      s[pp] = exp2f(s[pp] - msub);
-      lsum += s[pp];
-    }
-    l_run = l_run * alpha + lsum;
-    m_run = m_new;
-#pragma unroll
-    for (int h = 0; h < R; ++h) {
-      const float a = __shfl_sync(0xffffffffu, alpha, h * (LPR / R));
-#pragma unroll
-      for (int e = 0; e < E / 2; ++e) {
-        acc[h][e].x *= a;
-        acc[h][e].y *= a;
+      for (int nn = 0; nn < NT / 2; ++nn) {
+        const int ch = 2 * nn + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sV + (ch >> 3) * K::BOX + swz(vrow, ch & 7), b0, b1, b2, b3);
+        mma_16816(o[2 * nn], pa, b0, b1);
+        mma_16816(o[2 * nn + 1], pa, b2, b3);
       }
     }
 
-    // ---- value mix
-#pragma unroll
-    for (int pp = 0; pp < NP; ++pp) {
-      const int rr = w * K::RW + pp * K::RPP + rip;
-      float ph[R];
-#pragma unroll
-      for (int h = 0; h < R; ++h)
-        ph[h] = __shfl_sync(0xffffffffu, s[pp], rip * LPR + h * (LPR / R));
-      if (rr < hd.nrows) {
-#pragma unroll
-        for (int i = 0; i < NC; ++i) {
-          const uint4 u = *reinterpret_cast<const uint4 *>(
-              sV + rr * D + 8 * (sub + LPR * i));
-          const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 vf = make_float2(bf16lo_to_f32(w4[j]), bf16hi_to_f32(w4[j]));
-#pragma unroll
-            for (int h = 0; h < R; ++h)
-              ffma2(acc[h][i * 4 + j], make_float2(ph[h], ph[h]), vf);
-          }
-        }
-      }
-    }
-
-    // ---- end of a lane segment: combine the four warps into one partial
+    // ---- end of a lane segment: combine the warps, then output or partial
     if (hd.flags & kLast) {
-      float l_tot = l_run;
+      float l_tot[2];
 #pragma unroll
-      for (int off = LPR; off < 32; off <<= 1)
-        l_tot += __shfl_xor_sync(0xffffffffu, l_tot, off);
-#pragma unroll
-      for (int h = 0; h < R; ++h)
-#pragma unroll
-        for (int e = 0; e < E / 2; ++e)
-#pragma unroll
-          for (int off = LPR; off < 32; off <<= 1) {
-            acc[h][e].x += __shfl_xor_sync(0xffffffffu, acc[h][e].x, off);
-            acc[h][e].y += __shfl_xor_sync(0xffffffffu, acc[h][e].y, off);
-          }
-      // Everyone is done reading this stage's K/V: reuse it as scratch.
-      __syncwarp();
-      if (lane == 0) mbar_arrive(comb);
-      mbar_wait(comb, comb_count & 1, &failed);
-      comb_count++;
-      float *sm_m = reinterpret_cast<float *>(base);
-      float *sm_l = sm_m + kComputeWarps * R;
-      float *sm_acc = sm_l + kComputeWarps * R;
-      if (rip == 0) {
-#pragma unroll
-        for (int h = 0; h < R; ++h)
-#pragma unroll
-          for (int i = 0; i < NC; ++i)
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<float2 *>(
-                  sm_acc + (w * R + h) * D + 8 * (sub + LPR * i) + 2 * j) =
-                  acc[h][i * 4 + j];
-        if (sub % (LPR / R) == 0) {
-          sm_m[w * R + h_lane] = m_run;
-          sm_l[w * R + h_lane] = l_tot;
-        }
+      for (int i = 0; i < 2; ++i) {
+        float l = l_run[i];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        l_tot[i] = l;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(comb);
-      mbar_wait(comb, comb_count & 1, &failed);
-      comb_count++;
-      const int tid = threadIdx.x;  // 0..127
-      for (int idx = tid; idx < R * D; idx += kComputeWarps * 32) {
+      // Every warp is done with this stage: reuse it as scratch.
+      csync(comb, comb_count, &failed);
+      float *sm_m = reinterpret_cast<float *>(base);   // [NWC][16]
+      float *sm_l = sm_m + NWC * 16;                     // [NWC][16]
+      float *sm_acc = sm_l + NWC * 16;                   // [NWC][R][D]
+      if (t == 0) {
+        sm_m[w * 16 + g] = m_run[0];
+        sm_l[w * 16 + g] = l_tot[0];
+        sm_m[w * 16 + g + 8] = m_run[1];
+        sm_l[w * 16 + g + 8] = l_tot[1];
+      }
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        if (g < R)
+          *reinterpret_cast<float2 *>(sm_acc + (w * R + g) * D + n * 8 + 2 * t) =
+              make_float2(o[n][0], o[n][1]);
+        if (g + 8 < R)
+          *reinterpret_cast<float2 *>(sm_acc + (w * R + g + 8) * D + n * 8 + 2 * t) =
+              make_float2(o[n][2], o[n][3]);
+      }
+      csync(comb, comb_count, &failed);
+      const int L = hd.lane, b = L / p.VL, vl = L % p.VL;
+      const int h0 = (vl / p.nsub) * p.r + (vl % p.nsub) * R;
+      const int rc = min(R, p.r - (vl % p.nsub) * R);
+      __nv_bfloat16 *out = p.o + ((size_t)b * p.Hq + h0) * D;
+      for (int idx = threadIdx.x; idx < R * D; idx += NWC * 32) {
         const int h = idx / D, f = idx - (idx / D) * D;
         float mm = -INFINITY;
 #pragma unroll
-        for (int ww = 0; ww < kComputeWarps; ++ww) mm = fmaxf(mm, sm_m[ww * R + h]);
+        for (int ww = 0; ww < NWC; ++ww) mm = fmaxf(mm, sm_m[ww * 16 + h]);
         float a = 0.f, l = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kComputeWarps; ++ww) {
-          const float mw = sm_m[ww * R + h];
+        for (int ww = 0; ww < NWC; ++ww) {
+          const float mw = sm_m[ww * 16 + h];
           const float e = mw == -INFINITY ? 0.f : exp2f(mw - mm);
           a += e * sm_acc[(ww * R + h) * D + f];
-          l += e * sm_l[ww * R + h];
+          l += e * sm_l[ww * 16 + h];
         }
-        p.acc[((size_t)hd.slot * R + h) * D + f] = a;
-        if (f == 0) p.ml[(size_t)hd.slot * R + h] = make_float2(mm, l);
+        if (hd.np == 1) {
+          if (h < rc) out[idx] = __float2bfloat16_rn(a / l);
+        } else {
+          p.acc[((size_t)hd.slot * R + h) * D + f] = a;
+          if (f == 0) p.ml[(size_t)hd.slot * R + h] = make_float2(mm, l);
+        }
+      }
+      if (hd.np > 1) {
+        // Publish the partial, count it; the last CTA of the lane merges.
+        __threadfence();
+        csync(comb, comb_count, &failed);
+        if (threadIdx.x == 0)
+          merge_flag = (atomicAdd(&p.counters[L], 1) == hd.np - 1) ? 1 : 0;
+        csync(comb, comb_count, &failed);
+        if (merge_flag) {
+          __threadfence();
+          merge_lane<D, R>(p, L, hd.c0, hd.np, out, rc, sm_m, comb, comb_count, &failed);
+        }
       }
     }
     __syncwarp();
@@ -471,59 +562,45 @@ __device__ void consumer(const Params &p, unsigned char *smem,
 }
 
 template <int D, int R>
-__global__ void __launch_bounds__(kThreads, 2) split_kernel(const Params p) {
+__global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
+    split_kernel(const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const Params p) {
   using K = Cfg<D, R>;
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ unsigned char smem_raw[];
   __shared__ StageHdr hdrs[K::STAGES];
   __shared__ __align__(8) uint64_t full[K::STAGES], empty[K::STAGES], comb;
+  __shared__ int merge_flag;
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int s = 0; s < K::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kComputeWarps);
+      mbar_init(&empty[s], K::NWC);
     }
-    mbar_init(&comb, kComputeWarps);
+    mbar_init(&comb, K::NWC);
     fence_mbar_init();
   }
-  __syncthreads();
-  if ((threadIdx.x >> 5) == kComputeWarps)
-    producer<D, R>(p, smem, hdrs, full, empty);
-  else
-    consumer<D, R>(p, smem, hdrs, full, empty, &comb);
-}
-
-// Merge the partials of one virtual lane: grid (VL, B), 128 threads.
-template <int D, int R>
-__global__ void __launch_bounds__(128) merge_kernel(const Params p) {
-  const int vl = blockIdx.x, b = blockIdx.y;
-  const int L = b * p.VL + vl;
-  const int g = vl / p.nsub, sub = vl % p.nsub;
-  const int h0 = g * p.r + sub * R;
-  const int rc = min(R, p.r - sub * R);
-  __nv_bfloat16 *o = p.o + ((size_t)b * p.Hq + h0) * D;
-  const int n = p.seq_lens[b];
-  const bool ok = p.hdr->valid != 0 && n > 0;
-  if (!ok) {
-    for (int idx = threadIdx.x; idx < rc * D; idx += blockDim.x)
-      o[idx] = __float2bfloat16_rn(0.f);
-    return;
+  // Every length must lie in [0, C]; otherwise the call writes only zeros.
+  int bad_local = 0;
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const int n = p.seq_lens[b];
+    bad_local |= (n < 0 || n > p.C);
   }
-  const long long len = eligible(n, p.window);
-  const long long SL = p.lane_start[L];
-  const long long per = p.hdr->per;
-  const int c0 = (int)(SL / per), c1 = (int)((SL + len - 1) / per);
-  for (int idx = threadIdx.x; idx < rc * D; idx += blockDim.x) {
-    const int h = idx / D, f = idx - (idx / D) * D;
-    float mm = -INFINITY;
-    for (int c = c0; c <= c1; ++c) mm = fmaxf(mm, p.ml[(size_t)(L + c) * R + h].x);
-    float num = 0.f, den = 0.f;
-    for (int c = c0; c <= c1; ++c) {
-      const float2 ml = p.ml[(size_t)(L + c) * R + h];
-      const float e = ml.x == -INFINITY ? 0.f : exp2f(ml.x - mm);
-      num += e * p.acc[((size_t)(L + c) * R + h) * D + f];
-      den += e * ml.y;
+  const bool bad = __syncthreads_or(bad_local) != 0;
+  if (bad && blockIdx.x == 0 && threadIdx.x == 0) record_status(p.status, GQA_ERR_CAPACITY);
+  if ((threadIdx.x >> 5) == K::NWC) {
+    producer<D, R>(p, &tmK, &tmV, smem, hdrs, full, empty, bad);
+  } else {
+    // Rows of sequences with nothing to attend to (n_b = 0, or any invalid
+    // length) are zeros; CTA c takes batch rows c, c + G, ...
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+      if (!bad && p.seq_lens[b] > 0) continue;
+      __nv_bfloat16 *ob = p.o + (size_t)b * p.Hq * D;
+      for (int i = threadIdx.x; i < p.Hq * D / 8; i += K::NWC * 32)
+        reinterpret_cast<uint4 *>(ob)[i] = make_uint4(0, 0, 0, 0);
     }
-    o[idx] = __float2bfloat16_rn(num / den);
+    consumer<D, R>(p, smem, hdrs, full, empty, &comb, merge_flag);
   }
 }
 

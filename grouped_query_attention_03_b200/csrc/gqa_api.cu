@@ -24,7 +24,10 @@ namespace {
 using bf16 = __nv_bfloat16;
 
 constexpr int kMaxDecodeCtas = 1024;  // workspace is sized for this many
-constexpr int kDecodeMinRows = 128;   // rows below which a CTA is not split
+#ifndef GQA_DEC_MIN_ROWS
+#define GQA_DEC_MIN_ROWS 128
+#endif
+constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;  // smallest row range per CTA
 
 struct DeviceInfo {
   int sms = 0;
@@ -99,7 +102,7 @@ int next_pow2(int x) {
 
 // ------------------------------------------------------------ decode plan
 struct DecPlan {
-  int R = 1;     // heads stacked per CTA lane (power of two, <= 8)
+  int R = 1;     // heads stacked per CTA lane (power of two, <= 16)
   int nsub = 1;  // sub-groups per KV head
   int VL = 1;    // virtual lanes per batch row
 };
@@ -107,18 +110,21 @@ struct DecPlan {
 DecPlan decode_plan(int Hq, int Hkv) {
   DecPlan p;
   const int r = Hq / Hkv;
-  p.R = r >= 8 ? 8 : next_pow2(r);
+  p.R = r >= 16 ? 16 : next_pow2(r);
   p.nsub = (r + p.R - 1) / p.R;
   p.VL = Hkv * p.nsub;
   return p;
 }
 
 struct DecLayout {
-  size_t hdr = 0, lane_start = 0, ml = 0, acc = 0, total = 0;
+  size_t counters = 0, ml = 0, acc = 0, total = 0;
+  size_t counter_bytes = 0;
 };
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace: per-lane arrival counters (zeroed by each call), then the
+// (m, l) and acc partials, one slot per (lane, CTA) pair touching it.
 bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   const DecPlan pl = decode_plan(Hq, Hkv);
   int64_t lanes, slots, ml_elems, acc_elems;
@@ -127,9 +133,9 @@ bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   if (!elems(&ml_elems, {slots, pl.R})) return false;
   if (!elems(&acc_elems, {slots, pl.R, d})) return false;
   if (acc_elems > INT64_MAX / 8) return false;
-  L->hdr = 0;
-  L->lane_start = round256(sizeof(gqa::dec::WsHdr));
-  L->ml = L->lane_start + round256((size_t)lanes * sizeof(long long));
+  L->counters = 0;
+  L->counter_bytes = (size_t)lanes * sizeof(int);
+  L->ml = round256(L->counter_bytes);
   L->acc = L->ml + round256((size_t)ml_elems * sizeof(float2));
   L->total = L->acc + round256((size_t)acc_elems * sizeof(float));
   return true;
@@ -139,35 +145,44 @@ bool splitk_supported(gqa_dtype dtype, int d) {
   return dtype == GQA_BF16 && (d == 64 || d == 128);
 }
 
+// The split-K kernel addresses cache rows with 32-bit TMA coordinates.
+bool splitk_rows_ok(int B, int Hkv, int C) {
+  return (long long)B * Hkv * C < (1LL << 31);
+}
+
 template <int D, int R>
-gqa_status launch_splitk(const gqa::dec::Params &p, int sms, cudaStream_t st) {
+gqa_status launch_splitk(const gqa::dec::Params &p, const void *k_cache,
+                         const void *v_cache, int sms, cudaStream_t st) {
   using K = gqa::dec::Cfg<D, R>;
-  const int smem = K::STAGES * K::STAGE_BYTES;
+  CUtensorMap mk, mv;
+  const long long rows = (long long)p.B * p.Hkv * p.C;
+  if (!gqa::tma::make_bf16_map(&mk, k_cache, D, rows, 0, K::ROWS) ||
+      !gqa::tma::make_bf16_map(&mv, v_cache, D, rows, 0, K::ROWS))
+    return GQA_ERR_CUDA;
   static bool attr_done = false;  // per instantiation; benign race
   if (!attr_done) {
     if (cudaFuncSetAttribute(gqa::dec::split_kernel<D, R>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess) {
+                             K::SMEM) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;
     }
     attr_done = true;
   }
-  const int grid = std::min(kMaxDecodeCtas, 2 * sms);
-  gqa::dec::split_kernel<D, R><<<grid, gqa::dec::kThreads, smem, st>>>(p);
-  if (launch_status() != GQA_OK) return GQA_ERR_CUDA;
-  gqa::dec::merge_kernel<D, R><<<dim3(p.VL, p.B), 128, 0, st>>>(p);
+  const int grid = std::min(kMaxDecodeCtas, K::MIN_BLOCKS * sms);
+  gqa::dec::split_kernel<D, R><<<grid, K::THREADS, K::SMEM, st>>>(mk, mv, p);
   return launch_status();
 }
 
 template <int D>
-gqa_status dispatch_splitk_R(int R, const gqa::dec::Params &p, int sms,
-                             cudaStream_t st) {
+gqa_status dispatch_splitk_R(int R, const gqa::dec::Params &p, const void *kc,
+                             const void *vc, int sms, cudaStream_t st) {
   switch (R) {
-    case 1: return launch_splitk<D, 1>(p, sms, st);
-    case 2: return launch_splitk<D, 2>(p, sms, st);
-    case 4: return launch_splitk<D, 4>(p, sms, st);
-    case 8: return launch_splitk<D, 8>(p, sms, st);
+    case 1: return launch_splitk<D, 1>(p, kc, vc, sms, st);
+    case 2: return launch_splitk<D, 2>(p, kc, vc, sms, st);
+    case 4: return launch_splitk<D, 4>(p, kc, vc, sms, st);
+    case 8: return launch_splitk<D, 8>(p, kc, vc, sms, st);
+    case 16: return launch_splitk<D, 16>(p, kc, vc, sms, st);
   }
   return GQA_ERR_UNSUPPORTED;
 }
@@ -340,7 +355,7 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
   const bool aligned = aligned16(q) && aligned16(k_cache) &&
                        aligned16(v_cache) && aligned16(o);
   DeviceInfo di;
-  if (splitk_supported(dtype, d) && aligned) {
+  if (splitk_supported(dtype, d) && aligned && splitk_rows_ok(B, Hkv, C)) {
     DecLayout L;
     if (!decode_layout(B, Hq, Hkv, d, &L)) return GQA_ERR_OVERFLOW;
     if (!workspace || workspace_bytes < L.total ||
@@ -352,8 +367,6 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     gqa::dec::Params p;
     p.q = (const bf16 *)q;
-    p.kc = (const bf16 *)k_cache;
-    p.vc = (const bf16 *)v_cache;
     p.o = (bf16 *)o;
     p.seq_lens = seq_lens;
     p.B = B;
@@ -366,13 +379,16 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
     p.nsub = pl.nsub;
     p.VL = pl.VL;
     p.min_rows = kDecodeMinRows;
-    p.hdr = reinterpret_cast<gqa::dec::WsHdr *>(ws + L.hdr);
-    p.lane_start = reinterpret_cast<long long *>(ws + L.lane_start);
+    p.counters = reinterpret_cast<int *>(ws + L.counters);
     p.ml = reinterpret_cast<float2 *>(ws + L.ml);
     p.acc = reinterpret_cast<float *>(ws + L.acc);
     p.status = dev_status;
-    return d == 64 ? dispatch_splitk_R<64>(pl.R, p, di.sms, st)
-                   : dispatch_splitk_R<128>(pl.R, p, di.sms, st);
+    if (cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    return d == 64 ? dispatch_splitk_R<64>(pl.R, p, k_cache, v_cache, di.sms, st)
+                   : dispatch_splitk_R<128>(pl.R, p, k_cache, v_cache, di.sms, st);
   }
   if (Hq > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
   if ((s = device_info(&di)) != GQA_OK) return s;
