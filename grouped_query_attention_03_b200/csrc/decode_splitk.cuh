@@ -54,7 +54,7 @@ constexpr int kBR = 16;               // rows per compute warp per stage
 // Compute warps per CTA, CTAs per SM and ring depth (overridable when
 // building, for tuning).
 #ifndef GQA_DEC_NWC
-#define GQA_DEC_NWC 8
+#define GQA_DEC_NWC 7
 #endif
 #ifndef GQA_DEC_MIN_BLOCKS
 #define GQA_DEC_MIN_BLOCKS 1
@@ -278,76 +278,91 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
 __device__ __forceinline__ void csync(uint64_t *comb, int &count, bool *failed) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(comb);
-  mbar_wait(comb, count & 1, failed);
+  mbar_wait_spin(comb, count & 1, failed);
   count++;
 }
 
 // The last CTA to finish lane L merges its np partials (slots L+c0 ..):
 // m = max m_i, l = sum e^{m_i - m} l_i, o = sum e^{m_i - m} acc_i / l.
-// Runs on the compute warps; `scratch` holds 2 * R * NWC floats.
+// Warp 0 computes the per-head maxima, the weights e^{m_i - m} (into shared
+// memory) and the denominators; after one barrier every compute thread sums
+// its float4 groups of the output over the partials, issuing the partials'
+// loads in batches of 8 so they are in flight together (they were just
+// written by other CTAs and sit in L2).  `scratch` is the just-consumed
+// stage buffer.
 template <int D, int R>
 __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
-                           __nv_bfloat16 *out, int rc, float *scratch,
-                           uint64_t *comb, int &comb_count, bool *failed) {
+                                        __nv_bfloat16 *out, int rc, float *scratch,
+                                        uint64_t *comb, int &comb_count, bool *failed) {
   using K = Cfg<D, R>;
   constexpr int NT = K::NWC * 32;
-  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  constexpr int G4 = R * D / 4;                 // float4 groups of one partial
+  constexpr int QPT = (G4 + NT - 1) / NT;       // groups per thread
+  constexpr int CAP = (K::STAGE_BYTES / 4 - 64) / R;  // partials whose weights fit
+  const int t = threadIdx.x, lane = t & 31;
   const float2 *ml = p.ml + (size_t)(L + c0) * R;
-  float *red = scratch;            // [NWC][R]
-  float *msm = scratch + K::NWC * R;  // [R] max, then [R] denominators
-  float *lsm = msm + R;
-  const int h_t = t % R;  // NT is a multiple of R
-  float lm = -INFINITY;
-  for (int idx = t; idx < np * R; idx += NT) lm = fmaxf(lm, ml[idx].x);
-#pragma unroll
-  for (int off = 16; off >= R; off >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, off));
-  if (lane < R) red[w * R + lane] = lm;
-  csync(comb, comb_count, failed);
-  if (t < R) {
-    float m = red[t];
-#pragma unroll
-    for (int i = 1; i < K::NWC; ++i) m = fmaxf(m, red[i * R + t]);
-    msm[t] = m;
-  }
-  csync(comb, comb_count, failed);
-  const float mh = msm[h_t];
-  float ld = 0.f;
-  for (int idx = t; idx < np * R; idx += NT) {
-    const float2 v = ml[idx];
-    ld += v.x == -INFINITY ? 0.f : exp2f(v.x - mh) * v.y;
-  }
-#pragma unroll
-  for (int off = 16; off >= R; off >>= 1) ld += __shfl_xor_sync(0xffffffffu, ld, off);
-  if (lane < R) red[w * R + lane] = ld;
-  csync(comb, comb_count, failed);
-  if (t < R) {
-    float l = 0.f;
-#pragma unroll
-    for (int i = 0; i < K::NWC; ++i) l += red[i * R + t];
-    lsm[t] = l;
-  }
-  csync(comb, comb_count, failed);
-  // one float4 of output per thread and pass; loads of all partials issued
-  // back to back
   const float4 *acc4 = reinterpret_cast<const float4 *>(p.acc + (size_t)(L + c0) * R * D);
-  for (int q4 = t; q4 < R * D / 4; q4 += NT) {
-    const int h = q4 / (D / 4);
-    const float m = msm[h];
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int c = 0; c < np; ++c) {
-      const float mc = ml[c * R + h].x;
-      const float e = mc == -INFINITY ? 0.f : exp2f(mc - m);
-      const float4 a = acc4[(size_t)c * (R * D / 4) + q4];
-      x.x += e * a.x;
-      x.y += e * a.y;
-      x.z += e * a.z;
-      x.w += e * a.w;
+  float *lsm = scratch;        // [R] 1 / denominator
+  float *wsm = scratch + 64;   // [CAP][R] weights
+
+  float x[QPT][4];
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
+  for (int cs = 0; cs < np; cs += CAP) {
+    const int nc = min(CAP, np - cs);
+    if (t < 32) {
+      // Warp 0: lane j handles head j % R for partials j / R, j / R + 32/R..
+      // (R <= 16 divides 32).
+      const int h = lane % R;
+      float m = -INFINITY;
+      for (int idx = lane; idx < np * R; idx += 32) m = fmaxf(m, ml[idx].x);
+#pragma unroll
+      for (int off = 16; off >= R; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      float l = 0.f;
+      for (int idx = lane; idx < np * R; idx += 32) {
+        const float2 v = ml[idx];
+        const float e = v.x == -INFINITY ? 0.f : exp2f(v.x - m);
+        const int c = idx / R - cs;
+        if (c >= 0 && c < nc) wsm[c * R + h] = e;
+        l += e * v.y;
+      }
+#pragma unroll
+      for (int off = 16; off >= R; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      if (lane < R) lsm[lane] = 1.f / l;
     }
-    if (h < rc) {
-      const float inv = 1.f / lsm[h];
+    csync(comb, comb_count, failed);
+#pragma unroll
+    for (int i = 0; i < QPT; ++i) {
+      const int q4 = t + i * NT;
+      if (q4 < G4) {
+        const int h = q4 / (D / 4);
+        for (int j0 = 0; j0 < nc; j0 += 8) {
+          float4 a[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j0 + j < nc) a[j] = acc4[(size_t)(cs + j0 + j) * G4 + q4];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j0 + j < nc) {
+              const float e = wsm[(j0 + j) * R + h];
+              x[i][0] += e * a[j].x;
+              x[i][1] += e * a[j].y;
+              x[i][2] += e * a[j].z;
+              x[i][3] += e * a[j].w;
+            }
+        }
+      }
+    }
+    if (cs + CAP < np) csync(comb, comb_count, failed);  // wsm is rewritten
+  }
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) {
+    const int q4 = t + i * NT;
+    const int h = q4 / (D / 4);
+    if (q4 < G4 && h < rc) {
+      const float inv = lsm[h];
       *reinterpret_cast<uint2 *>(out + q4 * 4) =
-          make_uint2(pack_bf16(x.x * inv, x.y * inv), pack_bf16(x.z * inv, x.w * inv));
+          make_uint2(pack_bf16(x[i][0] * inv, x[i][1] * inv), pack_bf16(x[i][2] * inv, x[i][3] * inv));
     }
   }
 }

@@ -187,3 +187,4 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
 }
 }  // namespace tc
 }  // namespace gqa
+
