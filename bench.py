@@ -237,6 +237,13 @@ class PrefillStep:
         return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
                 "window": self.window, "permitted_pairs_per_head": self.pairs}
 
+    def kernel(self):
+        """The tensor-core kernel gqa_prefill dispatches to for this shape."""
+        w = self.w
+        if w.d in (64, 128) and (w.Hq // w.Hkv) % 2 == 0:
+            return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
+        return "pf::prefill_kernel (one query head per CTA)"
+
 
 def measure_prefill(w, window, device, reps, warmup):
     """Per-launch prefill time (CUDA events), L2 flushed between launches
@@ -259,7 +266,7 @@ def measure_prefill(w, window, device, reps, warmup):
     peaks, kind = measured_peaks()
     tflops = step.flops / (ms / 1e3) / 1e12
     return step, {
-        **step.describe(), "tflops": round(tflops, 2), "ms": round(ms, 4),
+        **step.describe(), "kernel": step.kernel(), "tflops": round(tflops, 2), "ms": round(ms, 4),
         "flops": step.flops, "frac_of_measured": round(tflops / peaks["bf16_tflops"], 4),
         "peak_kind": f"{kind} bf16 matmul (burst)", "frac_of_spec_2250": round(tflops / 2250.0, 4),
         "l2": "inputs exceed L2" if flush is None else "L2 flushed between launches"}
@@ -468,7 +475,7 @@ def run_gpu_prefill(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded normal rounded to bf16)",
         "config": dict(step.describe(), parallelism=f"replicas x{world}", l2=res["l2"]),
-        "roofline": {"bound": "tensor", "kernel": "pf::prefill_kernel",
+        "roofline": {"bound": "tensor", "kernel": step.kernel(),
                      "achieved": res["tflops"], "peak": peaks["bf16_tflops"],
                      "peak_kind": f"{kind} bf16 matmul (burst)", "unit": "TFLOP/s",
                      "frac": res["frac_of_measured"], "frac_of_spec_2250": res["frac_of_spec_2250"],

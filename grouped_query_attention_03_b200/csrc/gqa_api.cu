@@ -16,6 +16,7 @@
 #include "append.cuh"
 #include "common.cuh"
 #include "decode_splitk.cuh"
+#include "prefill_pair.cuh"
 #include "prefill_tc.cuh"
 #include "simt.cuh"
 
@@ -312,6 +313,11 @@ gqa_status gqa_prefill(gqa_dtype dtype, const void *q, const void *k,
   const float scale_log2 = scale * gqa::kLog2e;
   if (dtype == GQA_BF16 && gqa::pf::supported(d) && aligned16(q) &&
       aligned16(k) && aligned16(v) && aligned16(o)) {
+    // Heads of a group in pairs (one CTA per pair) when the group size is
+    // even; otherwise one head per CTA.
+    if (gqa::pf2::supported(d, Hq, Hkv))
+      return gqa::pf2::launch(q, k, v, o, seq_lens, B, Hq, Hkv, T, d, window,
+                              scale_log2, dev_status, st);
     return gqa::pf::launch(q, k, v, o, seq_lens, B, Hq, Hkv, T, d, window,
                            scale_log2, dev_status, di.sms, st);
   }

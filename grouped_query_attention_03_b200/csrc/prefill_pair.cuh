@@ -1,0 +1,447 @@
+// prefill_pair.cuh -- tcgen05 prefill for two query heads of one KV group.
+//
+// Same computation as prefill_tc.cuh ("Share key/value heads and make
+// context explicit", sections "Give each query head an explicit shared KV
+// head" and "Intersect the window with the context already permitted";
+// FlashAttention's running max/sum from "GQA, FlashAttention and the KV
+// cache"), organised so one CTA owns the same 128-row query tile of two
+// heads h0, h0+1 that share KV head g: every K and V tile is fetched once
+// and used by both (the GQA sharing applied to on-chip traffic), and the two
+// heads' softmax work overlaps the other head's tensor-core work.
+//
+//   warp 0      TMA producer: both Q tiles, then K_0, V_0, K_1, V_1, ... into
+//               a ring of NSLOT tile slots (128-byte swizzle, no multicast).
+//   warp 1      TMEM allocation (all 512 columns); lane 0 issues tcgen05.mma:
+//               S_A(0), S_B(0), then per KV tile j:
+//               O_A += P_A(j) V_j, S_A(j+1), O_B += P_B(j) V_j, S_B(j+1)
+//               so the tensor pipe runs one head while the other head's
+//               softmax warps work.
+//   warps 2-3   idle (they complete the first warpgroup, which hands most of
+//               its registers to the softmax warpgroups with setmaxnreg).
+//   warps 4-7   softmax of head A, warps 8-11 softmax of head B: thread = row
+//               (TMEM lane); the whole 128-score row is read from TMEM into
+//               registers at once, then row max, lazy O rescale, and bf16 P
+//               written to shared memory (K-major, 128-byte swizzle); O / l
+//               epilogue.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+d), O_B after it.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+#include "tma_host.cuh"
+
+namespace gqa {
+namespace pf2 {
+
+constexpr int kBM = 128, kBN = 128;
+constexpr int kThreads = 384;
+// Registers per thread after the split: the first warpgroup (producer, MMA
+// issuer, two idle warps) gives registers to the two softmax warpgroups.
+// 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * (launch registers).
+constexpr int kRegsLow = 80, kRegsHigh = 208;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int KB = D / 64;                  // 64-column blocks
+  static constexpr int BLK = kBM * 128;              // 128 rows x 128 B
+  static constexpr int TILE = KB * BLK;              // a Q, K or V tile
+  static constexpr int NSLOT = (D == 128) ? 3 : 6;   // K/V ring slots
+  static constexpr int OFF_QA = 0;
+  static constexpr int OFF_QB = TILE;
+  static constexpr int OFF_RING = 2 * TILE;
+  static constexpr int OFF_PA = OFF_RING + NSLOT * TILE;
+  static constexpr int P_BYTES = kBM * kBN * 2;
+  static constexpr int OFF_PB = OFF_PA + P_BYTES;
+  static constexpr int SMEM = OFF_PB + P_BYTES + 1024;
+  static constexpr uint32_t TM_O = 256;              // O_A column; O_B = TM_O + D
+};
+
+struct Params {
+  __nv_bfloat16 *o;
+  const int32_t *seq_lens;
+  int32_t *status;
+  int B, Hq, Hkv, T, window, num_mt, pairs;  // pairs = (Hq/Hkv) / 2
+  float scale_log2;
+};
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t full[6], empty[6];
+  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t mma_fin;
+  uint32_t tmem_base;
+};
+
+// Softmax and epilogue for one head (one 128-thread warpgroup, TMEM lanes
+// = query rows).  `hd` selects the head's S/O columns, P buffer, barriers.
+template <int D>
+__device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsigned char *smem,
+                                             uint32_t tmem, int hd, int b, int h, int m0,
+                                             int n_b, int j0, int nt, bool *failed) {
+  using K = Cfg<D>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q4 = warp & 3;
+  const int row = q4 * 32 + lane;
+  const int t = m0 + row;
+  const bool active = t < n_b;
+  const int lo_t = p.window > 0 ? max(0, t - (p.window - 1)) : 0;
+  const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+  const uint32_t tS = tmem + lane_base + hd * kBN;
+  const uint32_t tO = tmem + lane_base + K::TM_O + hd * D;
+  const float sc = p.scale_log2;
+  unsigned char *sP = smem + (hd ? K::OFF_PB : K::OFF_PA);
+  float m_run = -INFINITY, l_run = 0.f;
+  bool ok = true;
+  for (int j = 0; j < nt; ++j) {
+    const int kb = (j0 + j) * kBN;
+    if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[hd], j & 1, failed))) { ok = false; break; }
+    tc::fence_after_sync();
+    const bool edge = (kb + kBN - 1 > m0) || (p.window > 0 && kb < m0 + kBM - p.window);
+    // the whole row of scores: four TMEM loads, one wait
+    float s[kBN];
+#pragma unroll
+    for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(tS + c * 32, s + c * 32);
+    tc::tmem_wait_ld();
+    if (edge) {
+#pragma unroll
+      for (int i = 0; i < kBN; ++i) {
+        const int key = kb + i;
+        if (!(key <= t && key >= lo_t)) s[i] = -INFINITY;
+      }
+    }
+    // row maximum of s*scale (sc*max(s) for sc > 0, sc*min(s) otherwise)
+    float mx;
+    {
+      const bool neg = !(sc > 0.f);
+      float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (!neg) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) mc[i & 3] = fmaxf(mc[i & 3], s[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i) mc[i & 3] = fmaxf(mc[i & 3], s[i] == -INFINITY ? -INFINITY : -s[i]);
+      }
+      mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+    }
+    const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * fabsf(sc);
+    // O and P of this head are free once its previous PV has completed.
+    if (j >= 1) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (j - 1) & 1, failed))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+    }
+    if (j == 0) {
+      m_run = m_tile;
+    } else if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
+      const float m_new = fmaxf(m_run, m_tile);
+      const float alpha = m_new == m_run ? 1.f : exp2f(m_run - m_new);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        float ov[32];
+        tc::tmem_ld32(tO + c * 32, ov);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+        tc::tmem_st32(tO + c * 32, ov);
+      }
+      tc::tmem_wait_st();
+      l_run *= alpha;
+      m_run = m_new;
+    }
+    const float msub = m_run == -INFINITY ? 0.f : m_run;
+    // p = 2^(s*scale - m) -> bf16 P (K-major, 128-byte swizzle); packed
+    // fp32x2 for the scale-subtract and the row sum
+    float2 lsum2 = make_float2(0.f, 0.f);
+    const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-msub, -msub);
+#pragma unroll
+    for (int chunk = 0; chunk < kBN / 8; ++chunk) {  // 16-byte chunks of the P row
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = chunk * 8 + 2 * e;
+        const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
+        const float2 pv = make_float2(exp2f(x.x), exp2f(x.y));
+        lsum2 = fadd2v(lsum2, pv);
+        w4[e] = pack_bf16(pv.x, pv.y);
+      }
+      const int blk = chunk >> 3, cc = chunk & 7;
+      unsigned char *dst = sP + blk * K::BLK + (row >> 3) * 1024 + (row & 7) * 128 +
+                           ((cc ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    const float lsum = lsum2.x + lsum2.y;
+    l_run += lsum;
+    tc::fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars.p_full[hd]);
+  }
+
+  // epilogue: O / l in bf16, one row per thread; the whole warp reads TMEM
+  bool have = false;
+  if (nt > 0 && ok) {
+    have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (nt - 1) & 1, failed));
+    tc::fence_after_sync();
+  }
+  const float inv = (active && have && l_run > 0.f) ? 1.f / l_run : 0.f;
+  __nv_bfloat16 *orow = p.o + (((size_t)b * p.Hq + h) * p.T + min(t, p.T - 1)) * D;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    float ov[32];
+    if (have) {
+      tc::tmem_ld32(tO + c * 32, ov);
+      tc::tmem_wait_ld();
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ov[i] = 0.f;
+    }
+    if (t < p.T) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w4[i] = pack_bf16(ov[e * 8 + 2 * i] * inv, ov[e * 8 + 2 * i + 1] * inv);
+        *reinterpret_cast<uint4 *>(orow + c * 32 + e * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using K = Cfg<D>;
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ Bars bars;
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- which tile: longest causal rows first; then (b, g, pair)
+  const int per_mt = p.B * p.Hkv * p.pairs;
+  const int mt = p.num_mt - 1 - (int)(blockIdx.x / per_mt);
+  int rem = (int)(blockIdx.x % per_mt);
+  const int pr = rem % p.pairs;
+  rem /= p.pairs;
+  const int g = rem % p.Hkv, b = rem / p.Hkv;
+  const int r = p.Hq / p.Hkv;
+  const int h0 = g * r + 2 * pr;
+  const int m0 = mt * kBM;
+  int n_b = p.T;
+  if (p.seq_lens) {
+    n_b = p.seq_lens[b];
+    if (n_b < 0 || n_b > p.T) {
+      if (threadIdx.x == 0 && mt == 0 && g == 0 && pr == 0) record_status(p.status, GQA_ERR_CAPACITY);
+      n_b = 0;  // the whole sequence is written as zeros
+    }
+  }
+  int j0 = 0, nt = 0;
+  if (n_b > m0) {
+    const int lo = p.window > 0 ? max(0, m0 - (p.window - 1)) : 0;
+    const int hi = min(m0 + kBM - 1, n_b - 1);
+    j0 = lo / kBN;
+    nt = hi / kBN - j0 + 1;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < K::NSLOT; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars.s_full[h], 1);
+      mbar_init(&bars.p_full[h], 4);
+      mbar_init(&bars.o_done[h], 1);
+    }
+    mbar_init(&bars.mma_fin, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bars.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars.tmem_base;
+  bool failed = false;
+  if (warp >= 4) {
+    // ================================================= softmax warpgroups
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    const int hd = (warp - 4) / 4;  // warps 4-7: head A, 8-11: head B
+    softmax_head<D>(p, bars, smem, tmem, hd, b, h0 + hd, m0, n_b, j0, nt, &failed);
+  } else {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+  if (warp == 0) {
+    // ================================================= TMA producer
+    if (lane == 0 && nt > 0) {
+      tc::prefetch_tmap(&tmQ);
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(&bars.q_full, 2 * K::TILE);
+#pragma unroll
+      for (int c = 0; c < K::KB; ++c) {
+        tc::tma_load_3d(smem + K::OFF_QA + c * K::BLK, &tmQ, c * 64, m0, b * p.Hq + h0, &bars.q_full);
+        tc::tma_load_3d(smem + K::OFF_QB + c * K::BLK, &tmQ, c * 64, m0, b * p.Hq + h0 + 1, &bars.q_full);
+      }
+      int fills[K::NSLOT];
+#pragma unroll
+      for (int s = 0; s < K::NSLOT; ++s) fills[s] = 0;
+      for (int i = 0; i < 2 * nt; ++i) {  // K_0, V_0, K_1, V_1, ...
+        const int s = i % K::NSLOT;
+        if (i >= K::NSLOT && !mbar_wait(&bars.empty[s], ((i / K::NSLOT) - 1) & 1, &failed)) break;
+        const CUtensorMap *map = (i & 1) ? &tmV : &tmK;
+        const int row = (j0 + (i >> 1)) * kBN;
+        mbar_arrive_expect_tx(&bars.full[s], K::TILE);
+#pragma unroll
+        for (int c = 0; c < K::KB; ++c)
+          tc::tma_load_3d(smem + K::OFF_RING + s * K::TILE + c * K::BLK, map, c * 64, row,
+                          b * p.Hkv + g, &bars.full[s]);
+        fills[s]++;
+      }
+      // Never leave a TMA load in flight into an exiting CTA.
+      bool f2 = false;
+      mbar_wait(&bars.q_full, 0, &f2);
+#pragma unroll
+      for (int s = 0; s < K::NSLOT; ++s)
+        if (fills[s] > 0) mbar_wait(&bars.full[s], (fills[s] - 1) & 1, &f2);
+      failed |= f2;
+    }
+  } else if (warp == 1) {
+    // ================================================= MMA issuer
+    if (lane == 0 && nt > 0) {
+      constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
+      const uint32_t sQ[2] = {smem_u32(smem + K::OFF_QA), smem_u32(smem + K::OFF_QB)};
+      const uint32_t sP[2] = {smem_u32(smem + K::OFF_PA), smem_u32(smem + K::OFF_PB)};
+      auto slot_addr = [&](int i) { return smem_u32(smem + K::OFF_RING + (i % K::NSLOT) * K::TILE); };
+      auto wait_load = [&](int i) {
+        return mbar_wait(&bars.full[i % K::NSLOT], (i / K::NSLOT) & 1, &failed);
+      };
+      auto issue_s = [&](int hd, int j) {
+        const uint32_t sK = slot_addr(2 * j);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * K::BLK + (k & 3) * 32;
+          tc::mma_bf16_ss(tmem + hd * kBN, tc::sw128_desc(sQ[hd] + off, 16, 1024),
+                          tc::sw128_desc(sK + off, 16, 1024), idS, k > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(&bars.s_full[hd]);
+      };
+      auto issue_pv = [&](int hd, int j) {
+        const uint32_t sV = slot_addr(2 * j + 1);
+#pragma unroll
+        for (int k = 0; k < kBN / 16; ++k) {
+          const uint64_t da = tc::sw128_desc(sP[hd] + (k >> 2) * K::BLK + (k & 3) * 32, 16, 1024);
+          const uint64_t db = tc::sw128_desc(sV + k * 16 * 128, K::BLK, 1024);
+          tc::mma_bf16_ss(tmem + K::TM_O + hd * D, da, db, idO, (j > 0 || k > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(&bars.o_done[hd]);
+      };
+      bool ok = mbar_wait(&bars.q_full, 0, &failed) && wait_load(0);
+      if (ok) {
+        tc::fence_after_sync();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        tc::mma_commit(&bars.empty[0]);  // K_0
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        // head A: O_A += P_A(j) V_j, then S_A(j+1)
+        if (!mbar_wait(&bars.p_full[0], j & 1, &failed) || !wait_load(2 * j + 1)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(0, j);
+        if (j + 1 < nt) {
+          if (!wait_load(2 * j + 2)) { ok = false; break; }
+          tc::fence_after_sync();
+          issue_s(0, j + 1);
+        }
+        // head B: O_B += P_B(j) V_j (frees V_j), then S_B(j+1) (frees K_j+1)
+        if (!mbar_wait(&bars.p_full[1], j & 1, &failed)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(1, j);
+        tc::mma_commit(&bars.empty[(2 * j + 1) % K::NSLOT]);
+        if (j + 1 < nt) {
+          issue_s(1, j + 1);
+          tc::mma_commit(&bars.empty[(2 * j + 2) % K::NSLOT]);
+        }
+      }
+      // Drain: every MMA this thread issued has finished before TMEM is freed.
+      tc::mma_commit(&bars.mma_fin);
+      bool f2 = false;
+      mbar_wait(&bars.mma_fin, 0, &f2);
+      failed |= f2;
+    }
+  }
+  }
+
+  if (failed) record_status(p.status, kStatusTimeout);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host
+inline bool supported(int d, int Hq, int Hkv) {
+  return (d == 64 || d == 128) && (Hq / Hkv) % 2 == 0;
+}
+
+template <int D>
+gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
+                    const int32_t *lens, int B, int Hq, int Hkv, int T,
+                    int window, float scale_log2, int32_t *status,
+                    cudaStream_t st) {
+  using K = Cfg<D>;
+  CUtensorMap mq, mk, mv;
+  if (!tma::make_bf16_map(&mq, q, D, T, B * Hq, 128) ||
+      !tma::make_bf16_map(&mk, k, D, T, B * Hkv, 128) ||
+      !tma::make_bf16_map(&mv, v, D, T, B * Hkv, 128))
+    return GQA_ERR_CUDA;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(prefill_pair_kernel<D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             K::SMEM) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ERR_CUDA;
+    }
+    attr_done = true;
+  }
+  Params p;
+  p.o = (__nv_bfloat16 *)o;
+  p.seq_lens = lens;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = T;
+  p.window = window;
+  p.num_mt = (T + kBM - 1) / kBM;
+  p.pairs = (Hq / Hkv) / 2;
+  p.scale_log2 = scale_log2;
+  const long long grid = (long long)B * Hkv * p.pairs * p.num_mt;
+  if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
+  prefill_pair_kernel<D><<<(unsigned)grid, kThreads, K::SMEM, st>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+inline gqa_status launch(const void *q, const void *k, const void *v, void *o,
+                         const int32_t *lens, int B, int Hq, int Hkv, int T, int d,
+                         int window, float scale_log2, int32_t *status, cudaStream_t st) {
+  if (d == 64)
+    return launch_d<64>(q, k, v, o, lens, B, Hq, Hkv, T, window, scale_log2, status, st);
+  return launch_d<128>(q, k, v, o, lens, B, Hq, Hkv, T, window, scale_log2, status, st);
+}
+
+}  // namespace pf2
+}  // namespace gqa
