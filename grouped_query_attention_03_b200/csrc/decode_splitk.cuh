@@ -125,8 +125,7 @@ __device__ __forceinline__ int swz(int r, int ch) {
 template <int D, int R>
 __device__ void producer(const Params &p, const CUtensorMap *tmK,
                          const CUtensorMap *tmV, unsigned char *smem,
-                         StageHdr *hdrs, uint64_t *full, uint64_t *empty,
-                         bool bad) {
+                         StageHdr *hdrs, uint64_t *full, uint64_t *empty) {
   using K = Cfg<D, R>;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -145,14 +144,17 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     }
     return true;
   };
-  if (lane == 0) {
-    tc::prefetch_tmap(tmK);
-    tc::prefetch_tmap(tmV);
-  }
-
-  // Pass 1: the total eligible row count (lengths already validated).
+  // Pass 1: validity of every length and the total eligible row count.  The
+  // producer checks the lengths itself so that its first copies wait for one
+  // round trip to the lengths and no CTA-wide barrier.
   long long tot = 0;
-  for (int b = lane; b < p.B && !bad; b += 32) tot += eligible(p.seq_lens[b], p.window);
+  int bad_local = 0;
+  for (int b = lane; b < p.B; b += 32) {
+    const int n = p.seq_lens[b];
+    bad_local |= (n < 0 || n > p.C);
+    tot += eligible(max(n, 0), p.window);
+  }
+  const bool bad = __any_sync(0xffffffffu, bad_local) != 0;
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1)
     tot += __shfl_xor_sync(0xffffffffu, tot, off);
@@ -282,85 +284,86 @@ __device__ __forceinline__ void csync(uint64_t *comb, int &count, bool *failed) 
   count++;
 }
 
+// GPU-scope acquire-release fence: taken by one thread after a CTA barrier it
+// orders every store of the CTA before the thread's next global operation,
+// and (after an atomic that observed other CTAs' releases) their stores
+// before every later load of the CTA.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 // The last CTA to finish lane L merges its np partials (slots L+c0 ..):
 // m = max m_i, l = sum e^{m_i - m} l_i, o = sum e^{m_i - m} acc_i / l.
-// Warp 0 computes the per-head maxima, the weights e^{m_i - m} (into shared
-// memory) and the denominators; after one barrier every compute thread sums
-// its float4 groups of the output over the partials, issuing the partials'
-// loads in batches of 8 so they are in flight together (they were just
-// written by other CTAs and sit in L2).  `scratch` is the just-consumed
-// stage buffer.
+// Every compute thread owns QPT float4 groups of the lane's R x D output and
+// folds the partials in batches of NB with a running maximum, so the loads
+// of one batch (the partials' (m, l) pairs and accumulator groups, just
+// written by other CTAs and read through L2) are in flight together and a
+// lane of up to NB partials costs one round trip.
 template <int D, int R>
 __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
-                                        __nv_bfloat16 *out, int rc, float *scratch,
-                                        uint64_t *comb, int &comb_count, bool *failed) {
+                                        __nv_bfloat16 *out, int rc) {
   using K = Cfg<D, R>;
   constexpr int NT = K::NWC * 32;
   constexpr int G4 = R * D / 4;                 // float4 groups of one partial
   constexpr int QPT = (G4 + NT - 1) / NT;       // groups per thread
-  constexpr int CAP = (K::STAGE_BYTES / 4 - 64) / R;  // partials whose weights fit
-  const int t = threadIdx.x, lane = t & 31;
+  constexpr int NB = QPT == 1 ? 16 : (QPT == 2 ? 8 : 4);  // partials per batch
+  const int t = threadIdx.x;
   const float2 *ml = p.ml + (size_t)(L + c0) * R;
   const float4 *acc4 = reinterpret_cast<const float4 *>(p.acc + (size_t)(L + c0) * R * D);
-  float *lsm = scratch;        // [R] 1 / denominator
-  float *wsm = scratch + 64;   // [CAP][R] weights
 
-  float x[QPT][4];
+  float m[QPT], l[QPT], x[QPT][4];
 #pragma unroll
-  for (int i = 0; i < QPT; ++i) x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
-  for (int cs = 0; cs < np; cs += CAP) {
-    const int nc = min(CAP, np - cs);
-    if (t < 32) {
-      // Warp 0: lane j handles head j % R for partials j / R, j / R + 32/R..
-      // (R <= 16 divides 32).
-      const int h = lane % R;
-      float m = -INFINITY;
-      for (int idx = lane; idx < np * R; idx += 32) m = fmaxf(m, ml[idx].x);
-#pragma unroll
-      for (int off = 16; off >= R; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      float l = 0.f;
-      for (int idx = lane; idx < np * R; idx += 32) {
-        const float2 v = ml[idx];
-        const float e = v.x == -INFINITY ? 0.f : exp2f(v.x - m);
-        const int c = idx / R - cs;
-        if (c >= 0 && c < nc) wsm[c * R + h] = e;
-        l += e * v.y;
-      }
-#pragma unroll
-      for (int off = 16; off >= R; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      if (lane < R) lsm[lane] = 1.f / l;
-    }
-    csync(comb, comb_count, failed);
+  for (int i = 0; i < QPT; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.f;
+    x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
+  }
+  for (int j0 = 0; j0 < np; j0 += NB) {
+    float2 mv[QPT][NB];
+    float4 a[QPT][NB];
 #pragma unroll
     for (int i = 0; i < QPT; ++i) {
       const int q4 = t + i * NT;
-      if (q4 < G4) {
-        const int h = q4 / (D / 4);
-        for (int j0 = 0; j0 < nc; j0 += 8) {
-          float4 a[8];
+      const int h = q4 / (D / 4);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j0 + j < nc) a[j] = acc4[(size_t)(cs + j0 + j) * G4 + q4];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j0 + j < nc) {
-              const float e = wsm[(j0 + j) * R + h];
-              x[i][0] += e * a[j].x;
-              x[i][1] += e * a[j].y;
-              x[i][2] += e * a[j].z;
-              x[i][3] += e * a[j].w;
-            }
+      for (int j = 0; j < NB; ++j) {
+        if (q4 < G4 && j0 + j < np) {
+          mv[i][j] = __ldcg(ml + (size_t)(j0 + j) * R + h);
+          a[i][j] = __ldcg(acc4 + (size_t)(j0 + j) * G4 + q4);
+        } else {
+          mv[i][j] = make_float2(-INFINITY, 0.f);
+          a[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
     }
-    if (cs + CAP < np) csync(comb, comb_count, failed);  // wsm is rewritten
+#pragma unroll
+    for (int i = 0; i < QPT; ++i) {
+      float mb = m[i];
+#pragma unroll
+      for (int j = 0; j < NB; ++j) mb = fmaxf(mb, mv[i][j].x);
+      if (mb > m[i]) {
+        const float sc = m[i] == -INFINITY ? 0.f : exp2f(m[i] - mb);
+        l[i] *= sc;
+        x[i][0] *= sc; x[i][1] *= sc; x[i][2] *= sc; x[i][3] *= sc;
+        m[i] = mb;
+      }
+#pragma unroll
+      for (int j = 0; j < NB; ++j) {
+        const float e = mv[i][j].x == -INFINITY ? 0.f : exp2f(mv[i][j].x - m[i]);
+        l[i] += e * mv[i][j].y;
+        x[i][0] += e * a[i][j].x;
+        x[i][1] += e * a[i][j].y;
+        x[i][2] += e * a[i][j].z;
+        x[i][3] += e * a[i][j].w;
+      }
+    }
   }
 #pragma unroll
   for (int i = 0; i < QPT; ++i) {
     const int q4 = t + i * NT;
     const int h = q4 / (D / 4);
     if (q4 < G4 && h < rc) {
-      const float inv = lsm[h];
+      const float inv = 1.f / l[i];
       *reinterpret_cast<uint2 *>(out + q4 * 4) =
           make_uint2(pack_bf16(x[i][0] * inv, x[i][1] * inv), pack_bf16(x[i][2] * inv, x[i][3] * inv));
     }
@@ -557,16 +560,19 @@ __device__ void consumer(const Params &p, unsigned char *smem,
         }
       }
       if (hd.np > 1) {
-        // Publish the partial, count it; the last CTA of the lane merges.
-        __threadfence();
+        // Publish the partial and count it; the last CTA of the lane merges.
+        // After the barrier one thread's release fence covers the stores of
+        // the whole CTA; its acquire fence (when last) covers the loads of
+        // the merge, which every thread starts after the second barrier.
         csync(comb, comb_count, &failed);
-        if (threadIdx.x == 0)
-          merge_flag = (atomicAdd(&p.counters[L], 1) == hd.np - 1) ? 1 : 0;
-        csync(comb, comb_count, &failed);
-        if (merge_flag) {
-          __threadfence();
-          merge_lane<D, R>(p, L, hd.c0, hd.np, out, rc, sm_m, comb, comb_count, &failed);
+        if (threadIdx.x == 0) {
+          fence_acq_rel_gpu();
+          const int last = atomicAdd(&p.counters[L], 1) == hd.np - 1;
+          if (last) fence_acq_rel_gpu();
+          merge_flag = last;
         }
+        csync(comb, comb_count, &failed);
+        if (merge_flag) merge_lane<D, R>(p, L, hd.c0, hd.np, out, rc);
       }
     }
     __syncwarp();
@@ -587,6 +593,7 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
   __shared__ int merge_flag;
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int s = 0; s < K::STAGES; ++s) {
@@ -596,17 +603,23 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
     mbar_init(&comb, K::NWC);
     fence_mbar_init();
   }
-  // Every length must lie in [0, C]; otherwise the call writes only zeros.
-  int bad_local = 0;
-  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
-    const int n = p.seq_lens[b];
-    bad_local |= (n < 0 || n > p.C);
+  if (warp == K::NWC && lane == 0) {
+    tc::prefetch_tmap(&tmK);
+    tc::prefetch_tmap(&tmV);
   }
-  const bool bad = __syncthreads_or(bad_local) != 0;
-  if (bad && blockIdx.x == 0 && threadIdx.x == 0) record_status(p.status, GQA_ERR_CAPACITY);
-  if ((threadIdx.x >> 5) == K::NWC) {
-    producer<D, R>(p, &tmK, &tmV, smem, hdrs, full, empty, bad);
+  __syncthreads();
+  if (warp == K::NWC) {
+    producer<D, R>(p, &tmK, &tmV, smem, hdrs, full, empty);
   } else {
+    // Every length must lie in [0, C]; otherwise the call writes only zeros
+    // (each compute warp checks all lengths; so does the producer).
+    int bad_local = 0;
+    for (int b = lane; b < p.B; b += 32) {
+      const int n = p.seq_lens[b];
+      bad_local |= (n < 0 || n > p.C);
+    }
+    const bool bad = __any_sync(0xffffffffu, bad_local) != 0;
+    if (bad && blockIdx.x == 0 && threadIdx.x == 0) record_status(p.status, GQA_ERR_CAPACITY);
     // Rows of sequences with nothing to attend to (n_b = 0, or any invalid
     // length) are zeros; CTA c takes batch rows c, c + G, ...
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
