@@ -148,14 +148,22 @@ def decode_shape(w, window):
 
 class DecodeStep:
     """Append one token per sequence and decode it; the lengths are reset to
-    the cached count first so every step reads the same number of cells."""
+    the cached count first so every step reads the same number of cells.
 
-    def __init__(self, w, device, Hkv=None, window=None):
+    The step is one gqa_decode_append call (the append fused into the decode
+    kernel); run_separate() is the same step as gqa_cache_append followed by
+    gqa_decode, reported beside it."""
+
+    def __init__(self, w, device, Hkv=None, window=None, extra=0):
         from grouped_query_attention_03_b200 import gqa
         self.gqa = gqa
         self.w = w
         self.Hkv = Hkv or w.Hkv
-        self.window, self.cached, self.C = decode_shape(w, window)
+        self.window, self.cached, C = decode_shape(w, window)
+        # `extra` spare cells of capacity let the fused call run back to back
+        # (each call appends one cell) when it is timed alone
+        self.extra = extra
+        self.C = C + extra
         B, Hq, d = w.B, w.Hq, w.d
         C = self.C
         self.q, self.kc, self.vc = [t.to(device) for t in synthetic.decode_inputs(
@@ -167,27 +175,41 @@ class DecodeStep:
         self.o = torch.empty_like(self.q)
         self.ws = gqa.decode_workspace(self.q, self.kc)
         self.status = gqa.new_status(device)
-        n = np.array(self.cached) + 1
-        eff = np.minimum(n, self.window) if self.window else n
+        self.kv_bytes = self.kv_bytes_at(0)
         e = 2  # bf16
-        self.kv_bytes = int(2 * self.Hkv * eff.sum() * d * e)
         self.qo_bytes = int(2 * B * Hq * d * e)
-        self.append_bytes = int(2 * 2 * B * self.Hkv * d * e)
+        # the new K/V rows are read once (counted in kv_bytes) and written once
+        self.write_bytes = int(2 * B * self.Hkv * d * e)
         self.decode_bytes = self.kv_bytes + self.qo_bytes
-        self.step_bytes = self.decode_bytes + self.append_bytes
-        self.launches_per_step = 3  # append copy + commit, split (plus a 4-byte-per-lane memset)
+        self.step_bytes = self.decode_bytes + self.write_bytes
+        self.launches_per_step = 1  # the fused kernel (plus a lengths copy and a counter memset)
+        self.launches_separate = 3  # append copy + commit, split kernel
 
-    def run(self, ev=None):
+    def kv_bytes_at(self, grown):
+        """K+V bytes one step reads when `grown` cells were appended since the
+        lengths were reset (the window caps the cells read)."""
+        n = np.array(self.cached) + 1 + grown
+        eff = np.minimum(n, self.window) if self.window else n
+        return int(2 * self.Hkv * eff.sum() * self.w.d * 2)
+
+    def step_bytes_at(self, grown):
+        return self.kv_bytes_at(grown) + self.qo_bytes + self.write_bytes
+
+    def reset(self):
         self.lens.copy_(self.lens0, non_blocking=True)
-        self.gqa.cache_append(self.kc, self.vc, self.kn, self.vn, self.lens, status=self.status)
-        if ev is not None:
-            ev[0].record()
-        self.gqa.decode(self.q, self.kc, self.vc, self.lens, window=self.window, out=self.o,
-                        workspace=self.ws, status=self.status)
-        if ev is not None:
-            ev[1].record()
 
-    def run_decode(self):
+    def run_kernel(self):
+        self.gqa.decode_append(self.q, self.kc, self.vc, self.kn, self.vn, self.lens,
+                               window=self.window, out=self.o, workspace=self.ws,
+                               status=self.status)
+
+    def run(self):
+        self.reset()
+        self.run_kernel()
+
+    def run_separate(self):
+        self.reset()
+        self.gqa.cache_append(self.kc, self.vc, self.kn, self.vn, self.lens, status=self.status)
         self.gqa.decode(self.q, self.kc, self.vc, self.lens, window=self.window, out=self.o,
                         workspace=self.ws, status=self.status)
 
@@ -202,7 +224,7 @@ class DecodeStep:
     def describe(self):
         w = self.w
         d = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": self.Hkv, "d": w.d,
-             "window": self.window, "capacity": self.C,
+             "window": self.window, "capacity": self.C - self.extra,
              "keys_read_per_seq": "cached+1 (the appended token)",
              "l2": "inputs exceed the 126 MB L2; no flush" if self.kv_bytes > 126e6
              else "L2 flushed before every step by reading a 256 MB buffer (outside the timed interval)",
@@ -332,7 +354,8 @@ def run_gpu(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = workloads.BY_NAME[args.workload]
-    step = DecodeStep(w, device, Hkv=args.hkv, window=args.window)
+    K2 = min(args.steps, 100)  # back-to-back calls of the fused kernel alone
+    step = DecodeStep(w, device, Hkv=args.hkv, window=args.window, extra=K2 + 2)
     stream = torch.cuda.current_stream(device)
     need_flush = step.kv_bytes <= 126e6
     flush = make_flush(device) if need_flush else None
@@ -343,10 +366,18 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize(device)
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after warm-up")
-    # The step and the decode call alone, captured once and replayed: the
-    # timed region holds only device work (no per-call host overhead).
+    # The step (fused), the same step unfused, and the gqa_decode_append call
+    # alone, captured once and replayed: the timed regions hold only device
+    # work (no per-call host overhead).
     g_step = capture(step.run, device)
-    g_dec = capture(step.run_decode, device)
+    g_sep = capture(step.run_separate, device)
+    g_reset = capture(step.reset, device)
+    step.reset()
+    g_dec = capture(step.run_kernel, device)
+
+    def events(n):
+        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(n)]
 
     K = args.steps
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -354,25 +385,22 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize(device)
     with ClockSampler(local) as clocks:
         if flush is None:
+            # inputs exceed L2: steps back to back
             start.record(stream)
             for i in range(K):
                 g_step.replay()
             end.record(stream)
             torch.cuda.synchronize(device)
             total_ms = start.elapsed_time(end)
-            # the decode call alone, back to back (inputs exceed L2)
             start.record(stream)
             for i in range(K):
-                g_dec.replay()
+                g_sep.replay()
             end.record(stream)
             torch.cuda.synchronize(device)
-            dec_ms = [start.elapsed_time(end) / K]
+            sep_ms = start.elapsed_time(end)
         else:
             # L2 flushed (outside the timed intervals) before every step
-            step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                       for _ in range(K)]
-            dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                      for _ in range(K)]
+            step_ev, sep_ev = events(K), events(K)
             for i in range(K):
                 flush_l2(flush)
                 step_ev[i][0].record(stream)
@@ -380,13 +408,29 @@ def run_gpu(args, world, rank, local):
                 step_ev[i][1].record(stream)
             for i in range(K):
                 flush_l2(flush)
-                dec_ev[i][0].record(stream)
-                g_dec.replay()
-                dec_ev[i][1].record(stream)
+                sep_ev[i][0].record(stream)
+                g_sep.replay()
+                sep_ev[i][1].record(stream)
             torch.cuda.synchronize(device)
             total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
-            dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+            sep_ms = sum(a.elapsed_time(b) for a, b in sep_ev)
+        # the gqa_decode_append call alone, K2 calls in a row from the reset
+        # lengths (call i reads i more cells; its bytes are counted so)
+        g_reset.replay()
+        dec_ev = events(K2)
+        for i in range(K2):
+            if flush is not None:
+                flush_l2(flush)
+            dec_ev[i][0].record(stream)
+            g_dec.replay()
+            dec_ev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+        g_reset.replay()
+        torch.cuda.synchronize(device)
+    dec_bytes = [step.step_bytes_at(i) for i in range(K2)]
     barrier()
+    sep_ms = dist_max(sep_ms, device)
     total_ms = dist_max(total_ms, device)
     dec_avg_ms = statistics.mean(dec_ms)
 
@@ -420,7 +464,7 @@ def run_gpu(args, world, rank, local):
                          measure_prefill(workloads.PREFILL_B4_T1024, 256, device, 20, 3)[1]]
     peaks, peak_kind = measured_peaks()
     value = step.step_bytes * K * world / (total_ms / 1e3) / 1e9
-    achieved = step.decode_bytes / (dec_avg_ms / 1e3) / 1e9
+    achieved = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
     h2d = hq.numel() * hq.element_size() + hkn.numel() * hkn.element_size() * 2
     d2h = ho.numel() * ho.element_size()
     line = None
@@ -435,12 +479,18 @@ def run_gpu(args, world, rank, local):
             "dtype": "bf16", "data": "synthetic (seeded N(0,1) rounded to bf16)",
             "config": dict(step.describe(), parallelism=f"replicas x{world}"),
             "frac_of_spec_8TBs": round(value / SPEC_HBM_GBS, 4),
-            "roofline": {"bound": "hbm", "kernel": "gqa_decode (counter memset + dec::split_kernel with in-kernel merge)",
+            "separate_step": {"what": "gqa_cache_append then gqa_decode (same step, not fused)",
+                              "value": round(step.step_bytes * K * world / (sep_ms / 1e3) / 1e9, 2),
+                              "ms_per_step": round(sep_ms / K, 5),
+                              "gpu_launches_per_step": step.launches_separate},
+            "roofline": {"bound": "hbm",
+                         "kernel": "gqa_decode_append (counter memset + dec::split_kernel: fused append, in-kernel merge)",
                          "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
                          "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4),
                          "frac_of_spec_8TBs": round(achieved / SPEC_HBM_GBS, 4),
-                         "bytes_per_launch": step.decode_bytes,
+                         "bytes_per_launch": round(statistics.mean(dec_bytes)),
+                         "launches_timed": K2,
                          "avg_launch_us": round(dec_avg_ms * 1e3, 3),
                          "traffic": args.traffic},
             "e2e": {"value": round(step.step_bytes * K * world / (e2e_ms / 1e3) / 1e9, 2),

@@ -48,6 +48,9 @@ namespace gqa {
 namespace dec {
 
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+// Lengths of up to this many sequences are cached in shared memory (read
+// from global memory once per CTA); a fused append needs that.
+constexpr int kLensSmem = 4096;
 constexpr float kLazyRescale = 8.0f;  // log2 units
 constexpr int kBR = 16;               // rows per compute warp per stage
 
@@ -72,7 +75,10 @@ struct Cfg {
   static constexpr int KB = D / 64;                    // 64-column boxes
   static constexpr int BOX = ROWS * 128;               // bytes of one box
   static constexpr int KV_BYTES = KB * BOX;            // K (or V) per stage
-  static constexpr int QRAW = ((R * D * 2 + 1023) / 1024) * 1024;
+  // Query rows of the group, then the appended key and value rows (fused
+  // append), in one 1024-byte-aligned area after K and V.
+  static constexpr int NEWOFF = R * D * 2;
+  static constexpr int QRAW = ((R * D * 2 + 4 * D + 1023) / 1024) * 1024;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES + QRAW;
   static constexpr int STAGES = GQA_DEC_STAGES;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
@@ -92,7 +98,7 @@ struct StageHdr {
   int slot;   // partial slot (lane + CTA index)
   int c0;     // first CTA whose range touches the lane
   int np;     // number of CTAs whose ranges touch the lane
-  int pad;
+  int newrow; // stage row of the appended token (fused append), else -1
 };
 
 struct Params {
@@ -105,11 +111,26 @@ struct Params {
   int nsub;   // sub-groups of at most R heads per KV head
   int VL;     // virtual lanes per batch row = Hkv * nsub
   int min_rows;
-  int *counters;          // [B*VL], zero at kernel start
+  int *counters;          // [B*VL + 1], zero at kernel start; the last
+                          // entry counts finished CTAs (fused append)
   float2 *ml;             // [(grid + B*VL) * R]: (m, l)
   float *acc;             // [(grid + B*VL) * R * D]
   int32_t *status;
+  // Fused append: seq_lens holds the lengths before this step (add = 1),
+  // the step's key/value rows come from k_new / v_new ([B,Hkv,1,D]) and are
+  // written to the cache at cell seq_lens[b]; the last CTA to finish then
+  // advances every length by one.  add = 0: plain decode, seq_lens = n_b.
+  const __nv_bfloat16 *k_new, *v_new;
+  __nv_bfloat16 *k_cache, *v_cache;
+  int32_t *lens_out;
+  int add;
+  int lens_smem;  // 1: B <= kLensSmem, lengths cached in shared memory
 };
+
+// Keys of sequence b for this call (n_b, the appended token included).
+__device__ __forceinline__ int nlen(const Params &p, int b) {
+  return p.seq_lens[b] + p.add;
+}
 
 __device__ __forceinline__ int eligible(int n, int window) {
   return window > 0 ? min(n, window) : n;
@@ -125,7 +146,8 @@ __device__ __forceinline__ int swz(int r, int ch) {
 template <int D, int R>
 __device__ void producer(const Params &p, const CUtensorMap *tmK,
                          const CUtensorMap *tmV, unsigned char *smem,
-                         StageHdr *hdrs, uint64_t *full, uint64_t *empty) {
+                         StageHdr *hdrs, uint64_t *full, uint64_t *empty,
+                         int *s_len, int *s_bad, uint64_t *lens_ready) {
   using K = Cfg<D, R>;
   const int lane = threadIdx.x & 31;
   const int G = gridDim.x, c = blockIdx.x;
@@ -147,14 +169,22 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
   // Pass 1: validity of every length and the total eligible row count.  The
   // producer checks the lengths itself so that its first copies wait for one
   // round trip to the lengths and no CTA-wide barrier.
+  // With lens_smem the lengths are read from global memory here only and
+  // cached in shared memory for the rest of the CTA (the compute warps wait
+  // for them on lens_ready).
   long long tot = 0;
   int bad_local = 0;
   for (int b = lane; b < p.B; b += 32) {
-    const int n = p.seq_lens[b];
-    bad_local |= (n < 0 || n > p.C);
+    const int n = nlen(p, b);
+    if (p.lens_smem) s_len[b] = n;
+    bad_local |= (n < p.add || n > p.C);
     tot += eligible(max(n, 0), p.window);
   }
   const bool bad = __any_sync(0xffffffffu, bad_local) != 0;
+  if (lane == 0) *s_bad = bad ? 1 : 0;
+  __syncwarp();
+  mbar_arrive(lens_ready);
+  auto len_of = [&](int bb) { return p.lens_smem ? s_len[bb] : nlen(p, bb); };
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1)
     tot += __shfl_xor_sync(0xffffffffu, tot, off);
@@ -171,7 +201,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     for (int b0 = 0; b0 < p.B && b < 0; b0 += 32) {
       const int bb = b0 + lane;
       const long long x =
-          bb < p.B ? (long long)eligible(p.seq_lens[bb], p.window) * p.VL : 0;
+          bb < p.B ? (long long)eligible(len_of(bb), p.window) * p.VL : 0;
       long long incl = x;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -187,7 +217,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         cum += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
-    int n_b = p.seq_lens[b];
+    int n_b = len_of(b);
     int len = eligible(n_b, p.window);
     int lo = n_b - len;
     long long off0 = start - cum_b;
@@ -212,12 +242,14 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         h.slot = L + c;
         h.c0 = (int)(SL / per);
         h.np = (int)((SL + len - 1) / per) - h.c0 + 1;
+        h.newrow = (p.add && row + nrows == len) ? nrows - 1 : -1;
         const int g = vl / p.nsub, sub = vl % p.nsub;
         const int h0 = g * p.r + sub * R;
         const int rc = min(R, p.r - sub * R);
         const uint32_t qb = seg_first ? (uint32_t)rc * D * 2 : 0u;
+        const uint32_t nb = h.newrow >= 0 ? 4u * D : 0u;
         unsigned char *base = smem + (size_t)st * K::STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[st], 2 * K::KV_BYTES + qb);
+        mbar_arrive_expect_tx(&full[st], 2 * K::KV_BYTES + qb + nb);
         // Whole boxes are fetched; rows past the segment are never used.
         const int y = (b * p.Hkv + g) * p.C + lo + row;
 #pragma unroll
@@ -228,6 +260,13 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         if (seg_first)
           bulk_g2s(base + 2 * K::KV_BYTES, p.q + ((size_t)b * p.Hq + h0) * D, qb,
                    &full[st]);
+        if (nb) {
+          // The appended token's rows (its cache cell is not written yet).
+          const size_t src = ((size_t)b * p.Hkv + g) * D;
+          bulk_g2s(base + 2 * K::KV_BYTES + K::NEWOFF, p.k_new + src, 2 * D, &full[st]);
+          bulk_g2s(base + 2 * K::KV_BYTES + K::NEWOFF + 2 * D, p.v_new + src, 2 * D,
+                   &full[st]);
+        }
       }
       __syncwarp();
       fills[st]++;
@@ -244,13 +283,13 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
           int nb = -1;
           for (int b0 = b + 1; b0 < p.B && nb < 0 && pos < end; b0 += 32) {
             const int bb = b0 + lane;
-            const bool ne = bb < p.B && eligible(p.seq_lens[bb], p.window) > 0;
+            const bool ne = bb < p.B && eligible(len_of(bb), p.window) > 0;
             const unsigned m = __ballot_sync(0xffffffffu, ne);
             if (m) nb = b0 + __ffs(m) - 1;
           }
           if (nb < 0) break;
           b = nb;
-          n_b = p.seq_lens[b];
+          n_b = len_of(b);
           len = eligible(n_b, p.window);
           lo = n_b - len;
         }
@@ -424,13 +463,37 @@ __device__ void consumer(const Params &p, unsigned char *smem,
     }
 
     const int nv = hd.nrows - w * kBR;  // valid rows of this warp's 16
+    // Generic-proxy writes into the stage (below) are fenced against the
+    // TMA writes that refill it once it is released.
+    bool wrote = (hd.flags & kLast) != 0;
     if (nv < kBR && nv > 0) {
+      wrote = true;
       // Rows past the segment hold other data (maybe non-finite): zero this
       // warp's share of them in V so 0 * V stays 0.
       for (int idx = lane; idx < (kBR - nv) * (D / 8); idx += 32) {
         const int row = w * kBR + nv + idx / (D / 8), ch = idx % (D / 8);
         *reinterpret_cast<uint4 *>(base + K::KV_BYTES + (ch >> 3) * K::BOX +
                                    swz(row, ch & 7)) = make_uint4(0, 0, 0, 0);
+      }
+      __syncwarp();
+    }
+
+    if (hd.newrow >= 0 && (hd.newrow >> 4) == w) {
+      // This warp's rows hold the appended token, whose cache cell is not
+      // written yet: take its key and value from the step's input (staged
+      // with the stage), and write them to the cache (the first virtual lane
+      // of the KV head does).
+      wrote = true;
+      const int L = hd.lane, b = L / p.VL, vl = L % p.VL, g = vl / p.nsub;
+      const unsigned char *stg = base + 2 * K::KV_BYTES + K::NEWOFF;
+      const size_t dst = (((size_t)b * p.Hkv + g) * p.C + hd.cell0 + hd.newrow) * D;
+      for (int idx = lane; idx < 2 * (D / 8); idx += 32) {
+        const int isv = idx >= D / 8, ch = idx - isv * (D / 8);
+        const uint4 x = *reinterpret_cast<const uint4 *>(stg + idx * 16);
+        *reinterpret_cast<uint4 *>(base + isv * K::KV_BYTES + (ch >> 3) * K::BOX +
+                                   swz(hd.newrow, ch & 7)) = x;
+        if (vl % p.nsub == 0)
+          *reinterpret_cast<uint4 *>((isv ? p.v_cache : p.k_cache) + dst + ch * 8) = x;
       }
       __syncwarp();
     }
@@ -575,6 +638,7 @@ __device__ void consumer(const Params &p, unsigned char *smem,
         if (merge_flag) merge_lane<D, R>(p, L, hd.c0, hd.np, out, rc);
       }
     }
+    if (wrote) tc::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
     stage_count++;
@@ -590,9 +654,11 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
   extern __shared__ unsigned char smem_raw[];
   __shared__ StageHdr hdrs[K::STAGES];
   __shared__ __align__(8) uint64_t full[K::STAGES], empty[K::STAGES], comb;
-  __shared__ int merge_flag;
+  __shared__ int merge_flag, s_bad;
+  __shared__ __align__(8) uint64_t lens_ready;
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  int *s_len = reinterpret_cast<int *>(smem + K::STAGES * K::STAGE_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -601,6 +667,7 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
       mbar_init(&empty[s], K::NWC);
     }
     mbar_init(&comb, K::NWC);
+    mbar_init(&lens_ready, 32);
     fence_mbar_init();
   }
   if (warp == K::NWC && lane == 0) {
@@ -609,21 +676,35 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
   }
   __syncthreads();
   if (warp == K::NWC) {
-    producer<D, R>(p, &tmK, &tmV, smem, hdrs, full, empty);
+    producer<D, R>(p, &tmK, &tmV, smem, hdrs, full, empty, s_len, &s_bad, &lens_ready);
   } else {
-    // Every length must lie in [0, C]; otherwise the call writes only zeros
-    // (each compute warp checks all lengths; so does the producer).
-    int bad_local = 0;
-    for (int b = lane; b < p.B; b += 32) {
-      const int n = p.seq_lens[b];
-      bad_local |= (n < 0 || n > p.C);
+    // The producer validates every length (each must give n_b in [0, C];
+    // otherwise the call writes only zeros) and caches them.
+    bool failed = false;
+    const bool ok = mbar_wait(&lens_ready, 0, &failed);
+    const bool bad = !ok || s_bad != 0;
+    if (!ok && lane == 0) record_status(p.status, kStatusTimeout);
+    if (ok && bad && blockIdx.x == 0 && threadIdx.x == 0)
+      record_status(p.status, GQA_ERR_CAPACITY);
+    if (p.add && warp == 0) {
+      // Fused append: this CTA reads no length from global memory any more
+      // (the producer has its copy), so the last CTA to get here advances
+      // them, unless the call was refused.  This overlaps the first copies.
+      int last = 0;
+      if (lane == 0) {
+        fence_acq_rel_gpu();
+        last = atomicAdd(&p.counters[p.B * p.VL], 1) == (int)gridDim.x - 1;
+        if (last) fence_acq_rel_gpu();
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      __syncwarp();
+      if (last && !bad)
+        for (int b = lane; b < p.B; b += 32) p.lens_out[b] += 1;
     }
-    const bool bad = __any_sync(0xffffffffu, bad_local) != 0;
-    if (bad && blockIdx.x == 0 && threadIdx.x == 0) record_status(p.status, GQA_ERR_CAPACITY);
     // Rows of sequences with nothing to attend to (n_b = 0, or any invalid
     // length) are zeros; CTA c takes batch rows c, c + G, ...
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-      if (!bad && p.seq_lens[b] > 0) continue;
+      if (!bad && (p.lens_smem ? s_len[b] : nlen(p, b)) > 0) continue;
       __nv_bfloat16 *ob = p.o + (size_t)b * p.Hq * D;
       for (int i = threadIdx.x; i < p.Hq * D / 8; i += K::NWC * 32)
         reinterpret_cast<uint4 *>(ob)[i] = make_uint4(0, 0, 0, 0);

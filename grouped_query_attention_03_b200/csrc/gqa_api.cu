@@ -124,8 +124,9 @@ struct DecLayout {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace: per-lane arrival counters (zeroed by each call), then the
-// (m, l) and acc partials, one slot per (lane, CTA) pair touching it.
+// Workspace: per-lane arrival counters and one count of finished CTAs
+// (zeroed by each call), then the (m, l) and acc partials, one slot per
+// (lane, CTA) pair touching it.
 bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   const DecPlan pl = decode_plan(Hq, Hkv);
   int64_t lanes, slots, ml_elems, acc_elems;
@@ -135,7 +136,7 @@ bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   if (!elems(&acc_elems, {slots, pl.R, d})) return false;
   if (acc_elems > INT64_MAX / 8) return false;
   L->counters = 0;
-  L->counter_bytes = (size_t)lanes * sizeof(int);
+  L->counter_bytes = (size_t)(lanes + 1) * sizeof(int);
   L->ml = round256(L->counter_bytes);
   L->acc = L->ml + round256((size_t)ml_elems * sizeof(float2));
   L->total = L->acc + round256((size_t)acc_elems * sizeof(float));
@@ -164,14 +165,16 @@ gqa_status launch_splitk(const gqa::dec::Params &p, const void *k_cache,
   if (!attr_done) {
     if (cudaFuncSetAttribute(gqa::dec::split_kernel<D, R>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             K::SMEM) != cudaSuccess) {
+                             K::SMEM + gqa::dec::kLensSmem * 4) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;
     }
     attr_done = true;
   }
   const int grid = std::min(kMaxDecodeCtas, K::MIN_BLOCKS * sms);
-  gqa::dec::split_kernel<D, R><<<grid, K::THREADS, K::SMEM, st>>>(mk, mv, p);
+  // the lengths' shared-memory copy follows the stages
+  const int smem = K::SMEM + (p.lens_smem ? ((p.B * 4 + 15) & ~15) : 0);
+  gqa::dec::split_kernel<D, R><<<grid, K::THREADS, smem, st>>>(mk, mv, p);
   return launch_status();
 }
 
@@ -220,13 +223,14 @@ gqa_status launch_simt_decode(const void *q, const void *kc, const void *vc,
                               void *o, const int32_t *lens, int B, int Hq,
                               int Hkv, int C, int d, int window,
                               float scale_log2, int32_t *status,
-                              cudaStream_t st) {
+                              cudaStream_t st, const void *kn = nullptr,
+                              const void *vn = nullptr, int add = 0) {
   const dim3 grid(Hq, B);
   const int nf = (d + 31) / 32;
 #define GQA_DC(NF)                                                         \
   gqa::decode_simt_kernel<T, NF><<<grid, 32, 0, st>>>(                     \
       (const T *)q, (const T *)kc, (const T *)vc, (T *)o, lens, B, Hq, Hkv, \
-      C, d, window, scale_log2, status)
+      C, d, window, scale_log2, status, (const T *)kn, (const T *)vn, add)
   switch (nf) {
     case 1: GQA_DC(1); break;
     case 2: GQA_DC(2); break;
@@ -338,11 +342,23 @@ size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,
   return L.total;
 }
 
-gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
-                      const void *v_cache, void *o, const int32_t *seq_lens,
-                      int B, int Hq, int Hkv, int C, int d, int window,
-                      float scale, void *workspace, size_t workspace_bytes,
-                      int32_t *dev_status, gqa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused append's extra operands (null for a plain decode).
+struct AppendArgs {
+  void *k_cache, *v_cache;
+  const void *k_new, *v_new;
+  int32_t *seq_lens;
+};
+
+gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
+                       const void *v_cache, void *o, const int32_t *seq_lens,
+                       int B, int Hq, int Hkv, int C, int d, int window,
+                       float scale, void *workspace, size_t workspace_bytes,
+                       int32_t *dev_status, gqa_stream_t stream,
+                       const AppendArgs *ap) {
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
   if (B < 0 || C < 0) return GQA_ERR_SHAPE;
   gqa_status s = check_heads(Hq, Hkv, d);
@@ -355,13 +371,18 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
   if (B == 0) return GQA_OK;
   if (!q || !k_cache || !v_cache || !o || !seq_lens || !dev_status)
     return GQA_ERR_NULL;
+  if (ap && (!ap->k_new || !ap->v_new)) return GQA_ERR_NULL;
   if (d > GQA_MAX_HEAD_DIM) return GQA_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float scale_log2 = scale * gqa::kLog2e;
   const bool aligned = aligned16(q) && aligned16(k_cache) &&
-                       aligned16(v_cache) && aligned16(o);
+                       aligned16(v_cache) && aligned16(o) &&
+                       (!ap || (aligned16(ap->k_new) && aligned16(ap->v_new)));
   DeviceInfo di;
-  if (splitk_supported(dtype, d) && aligned && splitk_rows_ok(B, Hkv, C)) {
+  // A fused append needs the lengths cached in shared memory.
+  const bool lens_fit = !ap || B <= gqa::dec::kLensSmem;
+  if (splitk_supported(dtype, d) && aligned && splitk_rows_ok(B, Hkv, C) &&
+      lens_fit) {
     DecLayout L;
     if (!decode_layout(B, Hq, Hkv, d, &L)) return GQA_ERR_OVERFLOW;
     if (!workspace || workspace_bytes < L.total ||
@@ -389,6 +410,13 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
     p.ml = reinterpret_cast<float2 *>(ws + L.ml);
     p.acc = reinterpret_cast<float *>(ws + L.acc);
     p.status = dev_status;
+    p.k_new = ap ? (const bf16 *)ap->k_new : nullptr;
+    p.v_new = ap ? (const bf16 *)ap->v_new : nullptr;
+    p.k_cache = ap ? (bf16 *)ap->k_cache : nullptr;
+    p.v_cache = ap ? (bf16 *)ap->v_cache : nullptr;
+    p.lens_out = ap ? ap->seq_lens : nullptr;
+    p.add = ap ? 1 : 0;
+    p.lens_smem = B <= gqa::dec::kLensSmem ? 1 : 0;
     if (cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;
@@ -398,12 +426,49 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
   }
   if (Hq > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
   if ((s = device_info(&di)) != GQA_OK) return s;
-  if (dtype == GQA_F32)
-    return launch_simt_decode<float>(q, k_cache, v_cache, o, seq_lens, B, Hq,
-                                     Hkv, C, d, window, scale_log2,
-                                     dev_status, st);
-  return launch_simt_decode<bf16>(q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv,
-                                  C, d, window, scale_log2, dev_status, st);
+  // CUDA-core path: the decode reads the candidate rows from the input, then
+  // the append (same all-or-nothing length rule) writes them and advances
+  // the lengths.
+  const void *kn = ap ? ap->k_new : nullptr, *vn = ap ? ap->v_new : nullptr;
+  const int add = ap ? 1 : 0;
+  s = dtype == GQA_F32
+          ? launch_simt_decode<float>(q, k_cache, v_cache, o, seq_lens, B, Hq,
+                                      Hkv, C, d, window, scale_log2,
+                                      dev_status, st, kn, vn, add)
+          : launch_simt_decode<bf16>(q, k_cache, v_cache, o, seq_lens, B, Hq,
+                                     Hkv, C, d, window, scale_log2, dev_status,
+                                     st, kn, vn, add);
+  if (s != GQA_OK || !ap) return s;
+  return gqa_cache_append(dtype, ap->k_cache, ap->v_cache, ap->k_new,
+                          ap->v_new, ap->seq_lens, B, Hkv, C, d, 1, dev_status,
+                          stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
+                      const void *v_cache, void *o, const int32_t *seq_lens,
+                      int B, int Hq, int Hkv, int C, int d, int window,
+                      float scale, void *workspace, size_t workspace_bytes,
+                      int32_t *dev_status, gqa_stream_t stream) {
+  return decode_impl(dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, C, d,
+                     window, scale, workspace, workspace_bytes, dev_status,
+                     stream, nullptr);
+}
+
+gqa_status gqa_decode_append(gqa_dtype dtype, const void *q, void *k_cache,
+                             void *v_cache, const void *k_new,
+                             const void *v_new, void *o, int32_t *seq_lens,
+                             int B, int Hq, int Hkv, int C, int d, int window,
+                             float scale, void *workspace,
+                             size_t workspace_bytes, int32_t *dev_status,
+                             gqa_stream_t stream) {
+  const AppendArgs ap{k_cache, v_cache, k_new, v_new, seq_lens};
+  return decode_impl(dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, C, d,
+                     window, scale, workspace, workspace_bytes, dev_status,
+                     stream, &ap);
 }
 
 gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,

@@ -17,7 +17,8 @@ template <typename T, int NF>
 __device__ void attend_row_warp(const T *__restrict__ qrow,
                                 const T *__restrict__ klane,
                                 const T *__restrict__ vlane, int lo, int hi,
-                                int d, float scale_log2, T *__restrict__ orow) {
+                                int d, float scale_log2, T *__restrict__ orow,
+                                const T *kcand = nullptr, const T *vcand = nullptr) {
   const int lane = threadIdx.x & 31;
   float q[NF], acc[NF];
 #pragma unroll
@@ -32,7 +33,8 @@ __device__ void attend_row_warp(const T *__restrict__ qrow,
     float s = -INFINITY;
     const int nk = min(32, hi - j0 + 1);
     for (int jj = 0; jj < nk; ++jj) {
-      const T *kr = klane + (size_t)(j0 + jj) * d;
+      // Key `hi` may be a candidate row held outside the lane (fused append).
+      const T *kr = (kcand && j0 + jj == hi) ? kcand : klane + (size_t)(j0 + jj) * d;
       float part = 0.f;
 #pragma unroll
       for (int i = 0; i < NF; ++i) {
@@ -61,7 +63,7 @@ __device__ void attend_row_warp(const T *__restrict__ qrow,
     for (int i = 0; i < NF; ++i) acc[i] *= alpha;
     for (int jj = 0; jj < nk; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const T *vr = vlane + (size_t)(j0 + jj) * d;
+      const T *vr = (vcand && j0 + jj == hi) ? vcand : vlane + (size_t)(j0 + jj) * d;
 #pragma unroll
       for (int i = 0; i < NF; ++i) {
         const int f = lane + 32 * i;
@@ -125,19 +127,23 @@ __global__ void __launch_bounds__(128)
 // Decode: grid (Hq, B), 32 threads; the query sits at cell n_b - 1 and
 // reads cells [max(0, n_b - w), n_b) of the shared cache lane.  An invalid
 // length anywhere zeroes the whole output (every warp checks every length).
+// With add = 1 (fused append) seq_lens holds the lengths before the step,
+// n_b = seq_lens[b] + 1, and cell n_b - 1 is read from kn / vn
+// ([B,Hkv,1,d]) instead of the cache, which is written afterwards.
 template <typename T, int NF>
 __global__ void __launch_bounds__(32)
     decode_simt_kernel(const T *__restrict__ q, const T *__restrict__ kc,
                        const T *__restrict__ vc, T *__restrict__ o,
                        const int32_t *__restrict__ seq_lens, int B, int Hq,
                        int Hkv, int C, int d, int window, float scale_log2,
-                       int32_t *status) {
+                       int32_t *status, const T *kn = nullptr,
+                       const T *vn = nullptr, int add = 0) {
   const int h = blockIdx.x, b = blockIdx.y;
   T *orow = o + ((size_t)b * Hq + h) * d;
   bool bad = false;
   for (int i = threadIdx.x; i < B; i += 32) {
-    const int n = seq_lens[i];
-    bad |= (n < 0 || n > C);
+    const int n = seq_lens[i] + add;
+    bad |= (n < add || n > C);
   }
   if (__any_sync(0xffffffffu, bad)) {
     if (threadIdx.x == 0 && b == 0 && h == 0)
@@ -145,7 +151,7 @@ __global__ void __launch_bounds__(32)
     zero_row_warp<T, NF>(orow, d);
     return;
   }
-  const int n = seq_lens[b];
+  const int n = seq_lens[b] + add;
   if (n == 0) {
     zero_row_warp<T, NF>(orow, d);
     return;
@@ -154,8 +160,10 @@ __global__ void __launch_bounds__(32)
   const int pos = n - 1;
   const int lo = window > 0 ? max(0, pos - (window - 1)) : 0;
   const size_t lane_off = ((size_t)b * Hkv + g) * C * d;
+  const size_t cand = ((size_t)b * Hkv + g) * d;
   attend_row_warp<T, NF>(q + ((size_t)b * Hq + h) * d, kc + lane_off,
-                         vc + lane_off, lo, pos, d, scale_log2, orow);
+                         vc + lane_off, lo, pos, d, scale_log2, orow,
+                         add ? kn + cand : nullptr, add ? vn + cand : nullptr);
 }
 
 }  // namespace gqa

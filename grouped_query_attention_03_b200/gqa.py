@@ -27,7 +27,7 @@ STATUS_NAMES = {
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_prefill", "gqa_decode", "gqa_decode_workspace_bytes",
-           "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
+           "gqa_decode_append", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
            "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
            "gqa_version")
 
@@ -63,6 +63,8 @@ def _declare(L):
     L.gqa_prefill.restype = i32
     L.gqa_decode.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, sz, vp, vp]
     L.gqa_decode.restype = i32
+    L.gqa_decode_append.argtypes = [i32] + [vp] * 7 + [i32] * 6 + [f32, vp, sz, vp, vp]
+    L.gqa_decode_append.restype = i32
     L.gqa_decode_noalloc.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, vp]
     L.gqa_decode_noalloc.restype = i32
     L.gqa_decode_workspace_bytes.argtypes = [i32] * 6
@@ -189,6 +191,38 @@ def decode(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,
         _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
         workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
         "gqa_decode")
+    return out
+
+
+def decode_append(q, k_cache, v_cache, k_new, v_new, seq_lens, *, window=None, scale=None,
+                  out=None, workspace=None, status=None, stream=None):
+    """The decode step with its cache append fused in: seq_lens [B] int32
+    counts the cells cached BEFORE the step; k_new/v_new [B,Hkv,1,d] are the
+    step's key and value rows.  Attends over the cached cells plus the new
+    row, writes the new row at cell seq_lens[b] and advances seq_lens in
+    place (all-or-nothing on the device)."""
+    B, Hq, d = q.shape
+    Hkv, C = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, C, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    if k_new.shape != (B, Hkv, 1, d) or v_new.shape != k_new.shape:
+        raise ValueError("new K/V must be [B,Hkv,1,d]")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    if workspace is None:
+        workspace = decode_workspace(q, k_cache)
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_decode_append(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(k_new, "k_new", q.dtype, dev),
+        _ptr(v_new, "v_new", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
+        _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
+        workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
+        "gqa_decode_append")
     return out
 
 

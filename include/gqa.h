@@ -116,8 +116,10 @@ gqa_status gqa_prefill(gqa_dtype dtype, const void *q, const void *k,
  *            gqa_decode_workspace_bytes(...) bytes, 256-byte aligned; its
  *            contents need no initialisation and are not preserved
  *   dev_status device int32 (required)
- * bf16 with d in {64, 128}: split-K flash-decode (bulk-copy fed shared
- * memory ring, group heads stacked per CTA) plus a merge pass.
+ * bf16 with d in {64, 128}: split-K flash-decode (TMA-fed shared memory
+ * ring, group heads stacked as tensor-core tile rows); the last CTA to
+ * finish a lane merges that lane's partials.  Other d and fp32 run on CUDA
+ * cores.
  */
 gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
                       const void *v_cache, void *o, const int32_t *seq_lens,
@@ -129,6 +131,37 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
  * returned for invalid sizes, which gqa_decode then rejects. */
 size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,
                                   int C, int d);
+
+/*
+ * gqa_decode_append -- the decode step with its cache append fused in.
+ * [P1] "Extend the existing full and cached attention paths": the step's
+ * new key/value row is read from the input as a candidate and takes part in
+ * the scores before it is committed to the cache; the append refuses to
+ * exceed capacity and never partly advances.
+ *
+ * Same result as gqa_cache_append(t_new = 1) followed by gqa_decode, in one
+ * kernel for bf16 with d in {64, 128} (the candidate row never makes a round
+ * trip through the cache):
+ *   seq_lens device int32 [B], in/out: len_b = cells cached BEFORE the step,
+ *            each in [0, C-1]; the query sits at cell len_b and reads cells
+ *            [max(0, len_b + 1 - w), len_b + 1), the last one from k_new /
+ *            v_new.  After the call len_b has grown by one.
+ *   k_new, v_new [B,Hkv,1,d]  the step's key (rotated) and value rows,
+ *            written to cell len_b of k_cache / v_cache
+ *   workspace  gqa_decode_workspace_bytes(...) bytes, as for gqa_decode
+ *   everything else as for gqa_decode.
+ * If any len_b lies outside [0, C-1], *dev_status is set to
+ * GQA_ERR_CAPACITY, the output is zero, and neither the caches nor the
+ * lengths change.  Other d and fp32 run a CUDA-core decode that reads the
+ * candidate rows from k_new / v_new, followed by gqa_cache_append.
+ */
+gqa_status gqa_decode_append(gqa_dtype dtype, const void *q, void *k_cache,
+                             void *v_cache, const void *k_new,
+                             const void *v_new, void *o, int32_t *seq_lens,
+                             int B, int Hq, int Hkv, int C, int d, int window,
+                             float scale, void *workspace,
+                             size_t workspace_bytes, int32_t *dev_status,
+                             gqa_stream_t stream);
 
 /* Size of the fixed device array gqa_decode_noalloc uses as its workspace. */
 #define GQA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)

@@ -100,6 +100,16 @@ def _append(L, **kw):
                               a["B"], a["Hkv"], a["C"], a["d"], a["t_new"], a["status"], None)
 
 
+def _decode_append(L, **kw):
+    a = dict(dtype=1, q=FAKE, kc=FAKE, vc=FAKE, kn=FAKE, vn=FAKE, o=FAKE, lens=FAKE, B=1,
+             Hq=4, Hkv=2, C=8, d=64, window=-1, scale=0.125, ws=FAKE, wsb=1 << 30,
+             status=FAKE)
+    a.update(kw)
+    return L.gqa_decode_append(a["dtype"], a["q"], a["kc"], a["vc"], a["kn"], a["vn"], a["o"],
+                               a["lens"], a["B"], a["Hq"], a["Hkv"], a["C"], a["d"],
+                               a["window"], a["scale"], a["ws"], a["wsb"], a["status"], None)
+
+
 def test_prefill_host_refusals(L):
     assert _prefill(L, Hq=6, Hkv=4) == GROUPS
     assert _prefill(L, Hkv=0) == SHAPE
@@ -123,6 +133,18 @@ def test_decode_host_refusals(L):
     assert _decode(L, status=None) == NULL
     assert _decode(L, C=-1) == SHAPE
     assert _decode(L, B=0, q=None) == OK
+
+
+def test_decode_append_host_refusals(L):
+    assert _decode_append(L, Hq=3, Hkv=2) == GROUPS
+    assert _decode_append(L, window=0) == WINDOW
+    assert _decode_append(L, kn=None) == NULL
+    assert _decode_append(L, vn=None) == NULL
+    assert _decode_append(L, lens=None) == NULL
+    assert _decode_append(L, status=None) == NULL
+    assert _decode_append(L, C=-1) == SHAPE
+    assert _decode_append(L, ws=None) == 8
+    assert _decode_append(L, B=0, q=None, kn=None) == OK
 
 
 def test_append_host_refusals(L):

@@ -171,6 +171,7 @@ DECODE_EDGES = [
     (64, 4, 1, 40, 128, list(range(0, 40, 1)) + [40] * 24, None),
     (2, 4, 2, 50, 96, [50, 3], None),
     (2, 3, 1, 50, 32, [17, 50], 5),
+    (4200, 2, 1, 3, 128, [b % 4 for b in range(4200)], None),  # lengths read from global memory
 ]
 
 
