@@ -33,10 +33,10 @@
 // CUDA-core formulation cannot do that beyond one or two heads per row.
 // At the end of a lane segment the warps' states are combined through the
 // just-consumed stage buffer.  A lane covered by one CTA is written out
-// directly; otherwise the combined (m, l, acc) goes to the workspace and the
-// last CTA to finish that lane (a per-lane atomic counter, zeroed at the
-// start of every call) merges the lane's partials and writes bf16 output.
-// No CTA ever waits for another.
+// directly; otherwise the combined (m, l, acc) goes to the workspace and is
+// counted when the CTA's range ends (a per-lane atomic counter, zeroed at the
+// start of every call); the last CTA to count a lane merges the lane's
+// partials and writes bf16 output.  No CTA ever waits for another.
 #pragma once
 
 #include <cuda.h>
@@ -85,7 +85,12 @@ struct Cfg {
   static constexpr int KS = D / 16;                    // k-steps of 16 features
   static constexpr int NT = D / 8;                     // 8-feature output tiles
   static_assert(R <= 16, "one 16-row tile holds the stacked heads");
-  static_assert(NWC * (2 * 16 + R * D) * 4 <= STAGE_BYTES,
+  static_assert(NWC > 4, "two merges split the compute warps 4 / NWC-4");
+  // Row stride (floats) of the combine scratch: padded by 8 when it fits,
+  // so the warps' fragment stores hit distinct banks.
+  static constexpr int ACC_STRIDE =
+      NWC * (2 * 16 + R * (D + 8)) * 4 <= STAGE_BYTES ? D + 8 : D;
+  static_assert(NWC * (2 * 16 + R * ACC_STRIDE) * 4 <= STAGE_BYTES,
                 "combine scratch must fit in one stage");
   static_assert(STAGE_BYTES % 1024 == 0 && BOX % 1024 == 0, "swizzle alignment");
 };
@@ -251,11 +256,15 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         unsigned char *base = smem + (size_t)st * K::STAGE_BYTES;
         mbar_arrive_expect_tx(&full[st], 2 * K::KV_BYTES + qb + nb);
         // Whole boxes are fetched; rows past the segment are never used.
+        // The cache is streamed once: evict it from L2 first, so that the
+        // partials and outputs stay there.
         const int y = (b * p.Hkv + g) * p.C + lo + row;
+        const uint64_t pol = tc::l2_policy_evict_first();
 #pragma unroll
         for (int kb = 0; kb < K::KB; ++kb) {
-          tc::tma_load_2d(base + kb * K::BOX, tmK, kb * 64, y, &full[st]);
-          tc::tma_load_2d(base + K::KV_BYTES + kb * K::BOX, tmV, kb * 64, y, &full[st]);
+          tc::tma_load_2d_hint(base + kb * K::BOX, tmK, kb * 64, y, &full[st], pol);
+          tc::tma_load_2d_hint(base + K::KV_BYTES + kb * K::BOX, tmV, kb * 64, y, &full[st],
+                               pol);
         }
         if (seg_first)
           bulk_g2s(base + 2 * K::KV_BYTES, p.q + ((size_t)b * p.Hq + h0) * D, qb,
@@ -333,20 +342,17 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 
 // The last CTA to finish lane L merges its np partials (slots L+c0 ..):
 // m = max m_i, l = sum e^{m_i - m} l_i, o = sum e^{m_i - m} acc_i / l.
-// Every compute thread owns QPT float4 groups of the lane's R x D output and
+// Each of the NT threads (t = 0 .. NT-1) owns QPT float4 groups of the lane's R x D output and
 // folds the partials in batches of NB with a running maximum, so the loads
 // of one batch (the partials' (m, l) pairs and accumulator groups, just
 // written by other CTAs and read through L2) are in flight together and a
 // lane of up to NB partials costs one round trip.
-template <int D, int R>
+template <int D, int R, int NT>
 __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
-                                        __nv_bfloat16 *out, int rc) {
-  using K = Cfg<D, R>;
-  constexpr int NT = K::NWC * 32;
+                                        __nv_bfloat16 *out, int rc, int t) {
   constexpr int G4 = R * D / 4;                 // float4 groups of one partial
   constexpr int QPT = (G4 + NT - 1) / NT;       // groups per thread
-  constexpr int NB = QPT == 1 ? 16 : (QPT == 2 ? 8 : 4);  // partials per batch
-  const int t = threadIdx.x;
+  constexpr int NB = QPT == 1 ? 16 : (QPT == 2 ? 8 : (QPT <= 4 ? 4 : 2));  // per batch
   const float2 *ml = p.ml + (size_t)(L + c0) * R;
   const float4 *acc4 = reinterpret_cast<const float4 *>(p.acc + (size_t)(L + c0) * R * D);
 
@@ -430,6 +436,9 @@ __device__ void consumer(const Params &p, unsigned char *smem,
   float o[NT][4];          // O tile accumulators
   float m_run[2], l_run[2];  // head rows g and g + 8
   int stage_count = 0, comb_count = 0;
+  // Split lanes whose partial this CTA wrote, counted at the end (at most
+  // two: the first and the last segment of the range).
+  int pend_n = 0, pL0 = 0, pc0 = 0, pn0 = 0, pL1 = 0, pc1 = 0, pn1 = 0;
 
   while (true) {
     const int st = stage_count % K::STAGES;
@@ -581,7 +590,7 @@ __device__ void consumer(const Params &p, unsigned char *smem,
       csync(comb, comb_count, &failed);
       float *sm_m = reinterpret_cast<float *>(base);   // [NWC][16]
       float *sm_l = sm_m + NWC * 16;                     // [NWC][16]
-      float *sm_acc = sm_l + NWC * 16;                   // [NWC][R][D]
+      float *sm_acc = sm_l + NWC * 16;                   // [NWC][R][ACC_STRIDE]
       if (t == 0) {
         sm_m[w * 16 + g] = m_run[0];
         sm_l[w * 16 + g] = l_tot[0];
@@ -591,10 +600,10 @@ __device__ void consumer(const Params &p, unsigned char *smem,
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
         if (g < R)
-          *reinterpret_cast<float2 *>(sm_acc + (w * R + g) * D + n * 8 + 2 * t) =
+          *reinterpret_cast<float2 *>(sm_acc + (w * R + g) * K::ACC_STRIDE + n * 8 + 2 * t) =
               make_float2(o[n][0], o[n][1]);
         if (g + 8 < R)
-          *reinterpret_cast<float2 *>(sm_acc + (w * R + g + 8) * D + n * 8 + 2 * t) =
+          *reinterpret_cast<float2 *>(sm_acc + (w * R + g + 8) * K::ACC_STRIDE + n * 8 + 2 * t) =
               make_float2(o[n][2], o[n][3]);
       }
       csync(comb, comb_count, &failed);
@@ -602,46 +611,95 @@ __device__ void consumer(const Params &p, unsigned char *smem,
       const int h0 = (vl / p.nsub) * p.r + (vl % p.nsub) * R;
       const int rc = min(R, p.r - (vl % p.nsub) * R);
       __nv_bfloat16 *out = p.o + ((size_t)b * p.Hq + h0) * D;
-      for (int idx = threadIdx.x; idx < R * D; idx += NWC * 32) {
-        const int h = idx / D, f = idx - (idx / D) * D;
-        float mm = -INFINITY;
+      // Warp w combines head rows w, w + NWC, ...: lane j < NWC weighs warp
+      // j's state, the weights reach every lane by shuffles, and each lane
+      // sums D/32 features over the warps.
+      for (int h = w; h < R; h += NWC) {
+        const float mw = lane < NWC ? sm_m[lane * 16 + h] : -INFINITY;
+        float mm = mw;
 #pragma unroll
-        for (int ww = 0; ww < NWC; ++ww) mm = fmaxf(mm, sm_m[ww * 16 + h]);
-        float a = 0.f, l = 0.f;
+        for (int off = 16; off >= 1; off >>= 1)
+          mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, off));
+        const float e = mw == -INFINITY ? 0.f : exp2f(mw - mm);
+        float lsum = lane < NWC ? e * sm_l[lane * 16 + h] : 0.f;
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1)
+          lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+        float a[D / 32];
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k) a[k] = 0.f;
 #pragma unroll
         for (int ww = 0; ww < NWC; ++ww) {
-          const float mw = sm_m[ww * 16 + h];
-          const float e = mw == -INFINITY ? 0.f : exp2f(mw - mm);
-          a += e * sm_acc[(ww * R + h) * D + f];
-          l += e * sm_l[ww * 16 + h];
+          const float ew = __shfl_sync(0xffffffffu, e, ww);
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k)
+            a[k] += ew * sm_acc[(ww * R + h) * K::ACC_STRIDE + lane + 32 * k];
         }
         if (hd.np == 1) {
-          if (h < rc) out[idx] = __float2bfloat16_rn(a / l);
+          if (h < rc) {
+            const float inv = 1.f / lsum;
+#pragma unroll
+            for (int k = 0; k < D / 32; ++k)
+              out[h * D + lane + 32 * k] = __float2bfloat16_rn(a[k] * inv);
+          }
         } else {
-          p.acc[((size_t)hd.slot * R + h) * D + f] = a;
-          if (f == 0) p.ml[(size_t)hd.slot * R + h] = make_float2(mm, l);
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k)
+            p.acc[((size_t)hd.slot * R + h) * D + lane + 32 * k] = a[k];
+          if (lane == 0) p.ml[(size_t)hd.slot * R + h] = make_float2(mm, lsum);
         }
       }
-      if (hd.np > 1) {
-        // Publish the partial and count it; the last CTA of the lane merges.
-        // After the barrier one thread's release fence covers the stores of
-        // the whole CTA; its acquire fence (when last) covers the loads of
-        // the merge, which every thread starts after the second barrier.
-        csync(comb, comb_count, &failed);
-        if (threadIdx.x == 0) {
-          fence_acq_rel_gpu();
-          const int last = atomicAdd(&p.counters[L], 1) == hd.np - 1;
-          if (last) fence_acq_rel_gpu();
-          merge_flag = last;
+      // A partial is counted at the end of the CTA's range: nobody needs it
+      // sooner (the lane's other pieces end with their CTAs' ranges), and the
+      // warps go on to the next segment without waiting for the count.  A
+      // range has at most two split lanes, its first and its last.
+      if (hd.np > 1 && pend_n < 2) {
+        if (pend_n == 0) {
+          pL0 = L; pc0 = hd.c0; pn0 = hd.np;
+        } else {
+          pL1 = L; pc1 = hd.c0; pn1 = hd.np;
         }
-        csync(comb, comb_count, &failed);
-        if (merge_flag) merge_lane<D, R>(p, L, hd.c0, hd.np, out, rc);
+        pend_n++;
       }
     }
     if (wrote) tc::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
     stage_count++;
+  }
+  if (pend_n > 0) {
+    // Publish and count this CTA's partials; it merges each lane it is the
+    // last to finish.  After the barrier one thread's release fence covers
+    // the stores of the whole CTA; its acquire fence (when last) covers the
+    // loads of the merges, which every thread starts after the second
+    // barrier.
+    csync(comb, comb_count, &failed);
+    if (threadIdx.x == 0) {
+      fence_acq_rel_gpu();
+      const int o0 = atomicAdd(&p.counters[pL0], 1);
+      const int o1 = pend_n > 1 ? atomicAdd(&p.counters[pL1], 1) : 0;
+      const int flags = (o0 == pn0 - 1 ? 1 : 0) | (pend_n > 1 && o1 == pn1 - 1 ? 2 : 0);
+      if (flags) fence_acq_rel_gpu();
+      merge_flag = flags;
+    }
+    csync(comb, comb_count, &failed);
+    const int flags = merge_flag;
+    // Two merges run side by side (warps 0-3 and the rest), one runs on
+    // every compute warp.
+    constexpr int NA = 4 * 32, NBT = (NWC - 4) * 32;
+    const int i = flags == 3 ? (w < 4 ? 0 : 1) : (flags == 2 ? 1 : 0);
+    if (flags) {
+      const int L = i ? pL1 : pL0, b = L / p.VL, vl = L % p.VL;
+      const int h0 = (vl / p.nsub) * p.r + (vl % p.nsub) * R;
+      const int rc = min(R, p.r - (vl % p.nsub) * R);
+      __nv_bfloat16 *out = p.o + ((size_t)b * p.Hq + h0) * D;
+      if (flags != 3)
+        merge_lane<D, R, NWC * 32>(p, L, i ? pc1 : pc0, i ? pn1 : pn0, out, rc, threadIdx.x);
+      else if (w < 4)
+        merge_lane<D, R, NA>(p, L, pc0, pn0, out, rc, threadIdx.x);
+      else
+        merge_lane<D, R, NBT>(p, L, pc1, pn1, out, rc, threadIdx.x - NA);
+    }
   }
   if (failed && lane == 0) record_status(p.status, kStatusTimeout);
 }

@@ -26,7 +26,7 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kMaxDecodeCtas = 1024;  // workspace is sized for this many
 #ifndef GQA_DEC_MIN_ROWS
-#define GQA_DEC_MIN_ROWS 128
+#define GQA_DEC_MIN_ROWS 256
 #endif
 constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;  // smallest row range per CTA
 
