@@ -137,6 +137,14 @@ __device__ __forceinline__ int nlen(const Params &p, int b) {
   return p.seq_lens[b] + p.add;
 }
 
+// a / b for non-negative a and positive b, with the 32-bit divide when
+// both fit (the 64-bit one is a long software sequence).
+__device__ __forceinline__ long long udiv(long long a, long long b) {
+  if (((unsigned long long)a | (unsigned long long)b) < (1ull << 32))
+    return (long long)((unsigned)a / (unsigned)b);
+  return a / b;
+}
+
 __device__ __forceinline__ int eligible(int n, int window) {
   return window > 0 ? min(n, window) : n;
 }
@@ -194,7 +202,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
   for (int off = 16; off >= 1; off >>= 1)
     tot += __shfl_xor_sync(0xffffffffu, tot, off);
   const long long total = tot * p.VL;
-  long long per = (total + G - 1) / G;
+  long long per = udiv(total + G - 1, G);
   if (per < p.min_rows) per = p.min_rows;
   const long long start = (long long)c * per;
   const long long end = min(total, start + per);
@@ -226,7 +234,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     int len = eligible(n_b, p.window);
     int lo = n_b - len;
     long long off0 = start - cum_b;
-    int vl = (int)(off0 / len);
+    int vl = (int)udiv(off0, len);
     int row = (int)(off0 - (long long)vl * len);
     long long pos = start;
     bool seg_first = true;
@@ -245,8 +253,8 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         h.nrows = nrows;
         h.flags = (seg_first ? kFirst : 0) | (last ? kLast : 0);
         h.slot = L + c;
-        h.c0 = (int)(SL / per);
-        h.np = (int)((SL + len - 1) / per) - h.c0 + 1;
+        h.c0 = (int)udiv(SL, per);
+        h.np = (int)udiv(SL + len - 1, per) - h.c0 + 1;
         h.newrow = (p.add && row + nrows == len) ? nrows - 1 : -1;
         const int g = vl / p.nsub, sub = vl % p.nsub;
         const int h0 = g * p.r + sub * R;
