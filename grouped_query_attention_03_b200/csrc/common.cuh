@@ -174,6 +174,14 @@ __device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// 2^x with the special-function unit's instruction (ex2.approx.ftz.f32:
+// results below the normal range flush to zero, so 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 }  // namespace gqa
 
 namespace gqa {

@@ -40,7 +40,7 @@ constexpr int kThreads = 384;
 // Registers per thread after the split: the first warpgroup (producer, MMA
 // issuer, two idle warps) gives registers to the two softmax warpgroups.
 // 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * (launch registers).
-constexpr int kRegsLow = 80, kRegsHigh = 208;
+constexpr int kRegsLow = 72, kRegsHigh = 216;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -76,6 +76,49 @@ struct Bars {
   uint32_t tmem_base;
 };
 
+// O *= alpha for this thread's TMEM lane (the whole warp takes part).
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    float ov[32];
+    tc::tmem_ld32(tO + c * 32, ov);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+    tc::tmem_st32(tO + c * 32, ov);
+  }
+  tc::tmem_wait_st();
+}
+
+// p = 2^(s*scale - m) for this thread's row of kBN scores (special-function
+// unit; masked cells give exactly 0), written as bf16 P (K-major, 128-byte
+// swizzle, 16-byte chunks); returns the row sum.
+template <int D>
+__device__ __forceinline__ float emit_p(const float *s, float sc, float m, unsigned char *sP,
+                                        int row) {
+  using K = Cfg<D>;
+  float2 lsum2 = make_float2(0.f, 0.f);
+  const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
+#pragma unroll
+  for (int chunk = 0; chunk < kBN / 8; ++chunk) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = chunk * 8 + 2 * e;
+      const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
+      const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      lsum2 = fadd2v(lsum2, pv);
+      w4[e] = pack_bf16(pv.x, pv.y);
+    }
+    const int blk = chunk >> 3, cc = chunk & 7;
+    unsigned char *dst = sP + blk * K::BLK + (row >> 3) * 1024 + (row & 7) * 128 +
+                         ((cc ^ (row & 7)) << 4);
+    *reinterpret_cast<uint4 *>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+  return lsum2.x + lsum2.y;
+}
+
 // Softmax and epilogue for one head (one 128-thread warpgroup, TMEM lanes
 // = query rows).  `hd` selects the head's S/O columns, P buffer, barriers.
 template <int D>
@@ -106,6 +149,14 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(tS + c * 32, s + c * 32);
     tc::tmem_wait_ld();
+    // O and P of this head are free once its previous PV has completed.
+    if (j >= 1) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (j - 1) & 1, failed))) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+    }
     if (edge) {
 #pragma unroll
       for (int i = 0; i < kBN; ++i) {
@@ -123,59 +174,22 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
         for (int i = 0; i < kBN; ++i) mc[i & 3] = fmaxf(mc[i & 3], s[i]);
       } else {
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) mc[i & 3] = fmaxf(mc[i & 3], s[i] == -INFINITY ? -INFINITY : -s[i]);
+        for (int i = 0; i < kBN; ++i)
+          mc[i & 3] = fmaxf(mc[i & 3], s[i] == -INFINITY ? -INFINITY : -s[i]);
       }
       mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
     }
     const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * fabsf(sc);
-    // O and P of this head are free once its previous PV has completed.
-    if (j >= 1) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (j - 1) & 1, failed))) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-    }
     if (j == 0) {
       m_run = m_tile;
     } else if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
       const float m_new = fmaxf(m_run, m_tile);
       const float alpha = m_new == m_run ? 1.f : exp2f(m_run - m_new);
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        float ov[32];
-        tc::tmem_ld32(tO + c * 32, ov);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-        tc::tmem_st32(tO + c * 32, ov);
-      }
-      tc::tmem_wait_st();
+      rescale_o<D>(tO, alpha);
       l_run *= alpha;
       m_run = m_new;
     }
-    const float msub = m_run == -INFINITY ? 0.f : m_run;
-    // p = 2^(s*scale - m) -> bf16 P (K-major, 128-byte swizzle); packed
-    // fp32x2 for the scale-subtract and the row sum
-    float2 lsum2 = make_float2(0.f, 0.f);
-    const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-msub, -msub);
-#pragma unroll
-    for (int chunk = 0; chunk < kBN / 8; ++chunk) {  // 16-byte chunks of the P row
-      uint32_t w4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = chunk * 8 + 2 * e;
-        const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
-        const float2 pv = make_float2(exp2f(x.x), exp2f(x.y));
-        lsum2 = fadd2v(lsum2, pv);
-        w4[e] = pack_bf16(pv.x, pv.y);
-      }
-      const int blk = chunk >> 3, cc = chunk & 7;
-      unsigned char *dst = sP + blk * K::BLK + (row >> 3) * 1024 + (row & 7) * 128 +
-                           ((cc ^ (row & 7)) << 4);
-      *reinterpret_cast<uint4 *>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-    }
-    const float lsum = lsum2.x + lsum2.y;
+    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, sP, row);
     l_run += lsum;
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
