@@ -306,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = exp2f(fmaf(s[c * 8 + 2 * e], sc, -msub));
-          const float p1 = exp2f(fmaf(s[c * 8 + 2 * e + 1], sc, -msub));
+          const float p0 = ex2_approx(fmaf(s[c * 8 + 2 * e], sc, -msub));
+          const float p1 = ex2_approx(fmaf(s[c * 8 + 2 * e + 1], sc, -msub));
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           lsum += __low2float(pr) + __high2float(pr);
           w4[e] = *reinterpret_cast<const uint32_t *>(&pr);

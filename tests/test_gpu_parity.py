@@ -67,6 +67,8 @@ PREFILL_EDGES = [
     (torch.bfloat16, 1, 4, 4, 257, 64, 1000, None),
     (torch.bfloat16, 1, 16, 1, 129, 64, 128, [129]),
     (torch.bfloat16, 1, 2, 2, 96, 96, None, None),
+    (torch.bfloat16, 2, 6, 2, 300, 128, None, [300, 150]),   # group of 3: one head per CTA
+    (torch.bfloat16, 1, 3, 3, 513, 128, 200, None),          # MHA with a window
     (torch.bfloat16, 2, 6, 2, 50, 32, 7, [50, 1]),
     (torch.float32, 1, 3, 1, 65, 40, None, [64]),
     (torch.float32, 2, 8, 4, 31, 256, 5, None),
