@@ -61,7 +61,11 @@ struct Params {
   __nv_bfloat16 *o;
   const int32_t *seq_lens;
   int32_t *status;
-  int B, Hq, Hkv, T, window, num_mt;
+  int B, Hq, Hkv, window, num_mt;
+  int Tq;      // query rows per head (Q and O are [B,Hq,Tq,d])
+  int Tk;      // key rows per KV lane (K and V are [B,Hkv,Tk,d])
+  int cached;  // 0: prompt, query row t at position t, n_b = active rows;
+               // 1: queries after a cache, query row i at position n_b-Tq+i
   float scale_log2;
 };
 
@@ -92,18 +96,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int m0 = mt * kBM;
-  int n_b = p.T;
+  // n_b keys of sequence b; `rows` query rows produce output, the query
+  // row i sits at key position off + i; a0 = position of this tile's row 0.
+  int n_b = p.Tk;
   if (p.seq_lens) {
     n_b = p.seq_lens[b];
-    if (n_b < 0 || n_b > p.T) {
+    if (n_b < 0 || n_b > p.Tk || (p.cached && n_b < p.Tq)) {
       if (threadIdx.x == 0 && mt == 0 && h == 0) record_status(p.status, GQA_ERR_CAPACITY);
-      n_b = 0;  // the whole sequence is written as zeros
+      n_b = -1;  // the whole sequence is written as zeros
     }
   }
+  const int off = (p.cached && n_b >= 0) ? n_b - p.Tq : 0;
+  const int rows = n_b < 0 ? 0 : (p.cached ? p.Tq : n_b);
+  const int a0 = off + m0;
+  const int n_keys = max(n_b, 0);
   int j0 = 0, nt = 0;
-  if (n_b > m0) {
-    const int lo = p.window > 0 ? max(0, m0 - (p.window - 1)) : 0;
-    const int hi = min(m0 + kBM - 1, n_b - 1);
+  if (rows > m0) {
+    const int lo = p.window > 0 ? max(0, a0 - (p.window - 1)) : 0;
+    const int hi = min(a0 + kBM - 1, off + rows - 1);
     j0 = lo / kBN;
     nt = hi / kBN - j0 + 1;
   }
@@ -225,8 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================================= softmax warps
     const int q4 = warp & 3;                 // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;          // query row within the tile
-    const int t = m0 + row;                  // absolute query cell
-    const bool active = t < n_b;
+    const int t = a0 + row;                  // key position of this query row
+    const int qr = m0 + row;                 // its row in Q and O
+    const bool active = t < off + rows;
     const int lo_t = p.window > 0 ? max(0, t - (p.window - 1)) : 0;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const float sc = p.scale_log2;
@@ -250,8 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.s_free[sb]);
 
-      const bool edge = (kb + kBN - 1 > m0) ||
-                        (p.window > 0 && kb < m0 + kBM - p.window);
+      const bool edge = (kb + kBN - 1 > a0) ||
+                        (p.window > 0 && kb < a0 + kBM - p.window);
       if (edge) {
 #pragma unroll
         for (int c = 0; c < kBN; ++c) {
@@ -318,6 +329,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4 *>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
       l_run += lsum;
+      if (kb + kBN > n_keys) {
+        // Cells past the sequence in this V tile are not the sequence's (an
+        // unwritten cache cell may hold NaN): their p is 0, but 0 * NaN is
+        // not, so clear those rows (thread = row) before P V is issued.
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.v_full[sb], (j >> 1) & 1, &failed))) {
+          ok = false;
+          break;
+        }
+        if (kb + row >= n_keys) {
+          unsigned char *vrow = smem + K::OFF_V + sb * K::TILE + row * 128;
+#pragma unroll
+          for (int c = 0; c < K::KB; ++c)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4 *>(vrow + c * K::BLK + ch * 16) = make_uint4(0, 0, 0, 0);
+        }
+      }
       tc::fence_proxy_async_smem();
       tc::fence_before_sync();
       __syncwarp();
@@ -332,18 +360,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::fence_after_sync();
     }
     const float inv = (active && have && l_run > 0.f) ? 1.f / l_run : 0.f;
-    __nv_bfloat16 *orow = p.o + (((size_t)b * p.Hq + h) * p.T + min(t, p.T - 1)) * D;
+    __nv_bfloat16 *orow = p.o + (((size_t)b * p.Hq + h) * p.Tq + min(qr, p.Tq - 1)) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       float ov[32];
       if (have) {
         tc::tmem_ld32(tmem + lane_base + 256 + c * 32, ov);
         tc::tmem_wait_ld();
-      } else {
+      }
+      if (!have || !active) {  // inactive rows are exact zeros (their O may be NaN)
 #pragma unroll
         for (int i = 0; i < 32; ++i) ov[i] = 0.f;
       }
-      if (t < p.T) {
+      if (qr < p.Tq) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           uint32_t w4[4];
@@ -377,13 +406,13 @@ inline bool supported(int d) { return d == 64 || d == 128; }
 
 template <int D>
 gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
-                    const int32_t *lens, int B, int Hq, int Hkv, int T,
-                    int window, float scale_log2, int32_t *status,
+                    const int32_t *lens, int B, int Hq, int Hkv, int Tq, int Tk,
+                    int cached, int window, float scale_log2, int32_t *status,
                     cudaStream_t st) {
   using K = Cfg<D>;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, D, T, B * Hq) || !make_map(&mk, k, D, T, B * Hkv) ||
-      !make_map(&mv, v, D, T, B * Hkv))
+  if (!make_map(&mq, q, D, Tq, B * Hq) || !make_map(&mk, k, D, Tk, B * Hkv) ||
+      !make_map(&mv, v, D, Tk, B * Hkv))
     return GQA_ERR_CUDA;
   static bool attr_done = false;
   if (!attr_done) {
@@ -402,9 +431,11 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.T = T;
+  p.Tq = Tq;
+  p.Tk = Tk;
+  p.cached = cached;
   p.window = window;
-  p.num_mt = (T + kBM - 1) / kBM;
+  p.num_mt = (Tq + kBM - 1) / kBM;
   p.scale_log2 = scale_log2;
   const long long grid = (long long)B * Hq * p.num_mt;
   if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
@@ -412,14 +443,16 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// Prompt (cached = 0: Tq = Tk = T) or queries after a cache (cached = 1:
+// Tq new rows against Tk = capacity cells).
 inline gqa_status launch(const void *q, const void *k, const void *v, void *o,
-                         const int32_t *lens, int B, int Hq, int Hkv, int T,
-                         int d, int window, float scale_log2, int32_t *status,
-                         int /*sms*/, cudaStream_t st) {
+                         const int32_t *lens, int B, int Hq, int Hkv, int Tq, int Tk,
+                         int cached, int d, int window, float scale_log2, int32_t *status,
+                         cudaStream_t st) {
   if (d == 64)
-    return launch_d<64>(q, k, v, o, lens, B, Hq, Hkv, T, window, scale_log2,
+    return launch_d<64>(q, k, v, o, lens, B, Hq, Hkv, Tq, Tk, cached, window, scale_log2,
                         status, st);
-  return launch_d<128>(q, k, v, o, lens, B, Hq, Hkv, T, window, scale_log2,
+  return launch_d<128>(q, k, v, o, lens, B, Hq, Hkv, Tq, Tk, cached, window, scale_log2,
                        status, st);
 }
 

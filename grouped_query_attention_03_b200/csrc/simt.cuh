@@ -89,37 +89,42 @@ __device__ void zero_row_warp(T *orow, int d) {
   }
 }
 
-// Prefill: grid (ceil(T/4), Hq, B), 128 threads; warp w owns query cell
-// t = 4*blockIdx.x + w of head blockIdx.y in batch row blockIdx.z.
+// Prefill: grid (ceil(Tq/4), Hq, B), 128 threads; warp w owns query row
+// i = 4*blockIdx.x + w of head blockIdx.y in batch row blockIdx.z.  Q and O
+// are [B,Hq,Tq,d], K and V [B,Hkv,Tk,d].  cached = 0: a prompt (Tq = Tk),
+// row i at key position i, rows i >= n_b zero.  cached = 1: Tq new rows
+// after a cache of n_b cells (the new ones included), row i at position
+// n_b - Tq + i.
 template <typename T, int NF>
 __global__ void __launch_bounds__(128)
     prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                         const T *__restrict__ v, T *__restrict__ o,
                         const int32_t *__restrict__ seq_lens, int Hq, int Hkv,
-                        int T_len, int d, int window, float scale_log2,
-                        int32_t *status) {
-  const int t = blockIdx.x * 4 + (threadIdx.x >> 5);
+                        int Tq, int Tk, int cached, int d, int window,
+                        float scale_log2, int32_t *status) {
+  const int i = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int h = blockIdx.y, b = blockIdx.z;
-  if (t >= T_len) return;
+  if (i >= Tq) return;
   const int r = Hq / Hkv, g = h / r;
-  T *orow = o + (((size_t)b * Hq + h) * T_len + t) * d;
-  int n = T_len;
+  T *orow = o + (((size_t)b * Hq + h) * Tq + i) * d;
+  int n = Tk;
   if (seq_lens) {
     n = seq_lens[b];
-    if (n < 0 || n > T_len) {
-      if ((threadIdx.x & 31) == 0 && t == 0 && h == 0)
+    if (n < 0 || n > Tk || (cached && n < Tq)) {
+      if ((threadIdx.x & 31) == 0 && i == 0 && h == 0)
         record_status(status, GQA_ERR_CAPACITY);
       zero_row_warp<T, NF>(orow, d);
       return;
     }
   }
+  const int t = cached ? n - Tq + i : i;
   if (t >= n) {  // inactive padded query: zero output
     zero_row_warp<T, NF>(orow, d);
     return;
   }
   const int lo = window > 0 ? max(0, t - (window - 1)) : 0;
-  const size_t lane_off = ((size_t)b * Hkv + g) * T_len * d;
-  attend_row_warp<T, NF>(q + (((size_t)b * Hq + h) * T_len + t) * d,
+  const size_t lane_off = ((size_t)b * Hkv + g) * Tk * d;
+  attend_row_warp<T, NF>(q + (((size_t)b * Hq + h) * Tq + i) * d,
                          k + lane_off, v + lane_off, lo, t, d, scale_log2,
                          orow);
 }

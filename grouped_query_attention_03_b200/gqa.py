@@ -27,7 +27,7 @@ STATUS_NAMES = {
 
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_prefill", "gqa_decode", "gqa_decode_workspace_bytes",
-           "gqa_decode_append", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
+           "gqa_decode_append", "gqa_decode_multi", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
            "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
            "gqa_version")
 
@@ -65,6 +65,8 @@ def _declare(L):
     L.gqa_decode.restype = i32
     L.gqa_decode_append.argtypes = [i32] + [vp] * 7 + [i32] * 6 + [f32, vp, sz, vp, vp]
     L.gqa_decode_append.restype = i32
+    L.gqa_decode_multi.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 7 + [f32, vp, vp]
+    L.gqa_decode_multi.restype = i32
     L.gqa_decode_noalloc.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, vp]
     L.gqa_decode_noalloc.restype = i32
     L.gqa_decode_workspace_bytes.argtypes = [i32] * 6
@@ -223,6 +225,30 @@ def decode_append(q, k_cache, v_cache, k_new, v_new, seq_lens, *, window=None, s
         _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
         workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
         "gqa_decode_append")
+    return out
+
+
+def decode_multi(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,
+                 status=None, stream=None):
+    """t_new new query rows per sequence against the cache: q [B,Hq,t_new,d],
+    caches [B,Hkv,C,d], seq_lens [B] int32 counting the cached cells
+    including the t_new new ones (query row i sits at cell n_b - t_new + i)."""
+    B, Hq, t_new, d = q.shape
+    Hkv, C = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape != (B, Hkv, C, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("cache shape mismatch")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_decode_multi(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d, t_new,
+        _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
+        _stream(stream, dev)), "gqa_decode_multi")
     return out
 
 

@@ -163,6 +163,35 @@ gqa_status gqa_decode_append(gqa_dtype dtype, const void *q, void *k_cache,
                              size_t workspace_bytes, int32_t *dev_status,
                              gqa_stream_t stream);
 
+/*
+ * gqa_decode_multi -- t_new new query rows per sequence against the cache
+ * (multi-token decode, chunked prefill).  [P4] the implementation's
+ * tril(s - t) mask offset and [P3] "The important mask bug with a cache":
+ * the new rows are the LAST t_new of the n_b cached cells (append them
+ * first with gqa_cache_append), so query row i sits at cell
+ * p_i = n_b - t_new + i and reads cells [max(0, p_i - (w-1)), p_i] of its
+ * shared lane ([P1] "Intersect the window with the context already
+ * permitted").  t_new = 1 is gqa_decode; t_new = n_b is a causal prefill of
+ * the whole cache.
+ *
+ *   q        [B,Hq,t_new,d]  the new rows' queries (already rotated)
+ *   k_cache, v_cache [B,Hkv,C,d]  caches of capacity C
+ *   o        [B,Hq,t_new,d]  output
+ *   seq_lens device int32 [B], n_b in [t_new, C] (required)
+ *   dev_status device int32 (required)
+ * Cells past n_b are never used, whatever they hold.  A length outside
+ * [t_new, C] sets *dev_status to GQA_ERR_CAPACITY and writes that
+ * sequence's output as zeros.  t_new > C returns GQA_ERR_CAPACITY before
+ * anything is enqueued.  bf16 with d in {64, 128} runs the tcgen05 prefill
+ * kernels with the query rows offset by n_b - t_new; other d and fp32 run
+ * on CUDA cores.
+ */
+gqa_status gqa_decode_multi(gqa_dtype dtype, const void *q, const void *k_cache,
+                            const void *v_cache, void *o, const int32_t *seq_lens,
+                            int B, int Hq, int Hkv, int C, int d, int t_new,
+                            int window, float scale, int32_t *dev_status,
+                            gqa_stream_t stream);
+
 /* Size of the fixed device array gqa_decode_noalloc uses as its workspace. */
 #define GQA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 

@@ -110,6 +110,28 @@ def _decode_append(L, **kw):
                                a["window"], a["scale"], a["ws"], a["wsb"], a["status"], None)
 
 
+def _decode_multi(L, **kw):
+    a = dict(dtype=1, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lens=FAKE, B=1, Hq=4, Hkv=2, C=8, d=64,
+             t_new=2, window=-1, scale=0.125, status=FAKE)
+    a.update(kw)
+    return L.gqa_decode_multi(a["dtype"], a["q"], a["k"], a["v"], a["o"], a["lens"], a["B"],
+                              a["Hq"], a["Hkv"], a["C"], a["d"], a["t_new"], a["window"],
+                              a["scale"], a["status"], None)
+
+
+def test_decode_multi_host_refusals(L):
+    assert _decode_multi(L, Hq=3, Hkv=2) == GROUPS
+    assert _decode_multi(L, window=0) == WINDOW
+    assert _decode_multi(L, t_new=9) == CAPACITY
+    assert _decode_multi(L, t_new=-1) == SHAPE
+    assert _decode_multi(L, C=-1) == SHAPE
+    assert _decode_multi(L, lens=None) == NULL
+    assert _decode_multi(L, status=None) == NULL
+    assert _decode_multi(L, q=None) == NULL
+    assert _decode_multi(L, t_new=0, q=None) == OK
+    assert _decode_multi(L, B=0, q=None) == OK
+
+
 def test_prefill_host_refusals(L):
     assert _prefill(L, Hq=6, Hkv=4) == GROUPS
     assert _prefill(L, Hkv=0) == SHAPE
