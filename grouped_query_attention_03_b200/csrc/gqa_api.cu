@@ -193,16 +193,16 @@ gqa_status dispatch_splitk_R(int R, const gqa::dec::Params &p, const void *kc,
 
 template <typename T>
 gqa_status launch_simt_prefill(const void *q, const void *k, const void *v,
-                               void *o, const int32_t *lens, int B, int Hq,
-                               int Hkv, int Tq, int Tk, int cached, int d,
-                               int window, float scale_log2, int32_t *status,
-                               cudaStream_t st) {
+                               void *o, const int32_t *lens, const int32_t *seg,
+                               int B, int Hq, int Hkv, int Tq, int Tk, int cached,
+                               int d, int window, float scale_log2,
+                               int32_t *status, cudaStream_t st) {
   const dim3 grid((Tq + 3) / 4, Hq, B);
   const int nf = (d + 31) / 32;
 #define GQA_PF(NF)                                                        \
   gqa::prefill_simt_kernel<T, NF><<<grid, 128, 0, st>>>(                  \
-      (const T *)q, (const T *)k, (const T *)v, (T *)o, lens, Hq, Hkv,    \
-      Tq, Tk, cached, d, window, scale_log2, status)
+      (const T *)q, (const T *)k, (const T *)v, (T *)o, lens, seg, Hq,    \
+      Hkv, Tq, Tk, cached, d, window, scale_log2, status)
   switch (nf) {
     case 1: GQA_PF(1); break;
     case 2: GQA_PF(2); break;
@@ -266,6 +266,7 @@ const char *gqa_status_string(gqa_status s) {
     case GQA_ERR_CUDA: return "CUDA runtime error";
     case GQA_ERR_DEVICE: return "current device is not an sm_100 GPU";
     case GQA_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case GQA_ERR_SEGMENT: return "a packed segment start lies outside [0, t]";
   }
   return "unknown status";
 }
@@ -303,10 +304,10 @@ namespace {
 // a prompt (cached = 0, Tq = Tk = T) or new rows after a cache (cached = 1,
 // Tk = capacity, query row i at position n_b - Tq + i).
 gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
-                       const void *v, void *o, const int32_t *seq_lens, int B,
-                       int Hq, int Hkv, int Tq, int Tk, int cached, int d,
-                       int window, float scale, int32_t *dev_status,
-                       gqa_stream_t stream) {
+                       const void *v, void *o, const int32_t *seq_lens,
+                       const int32_t *seg, int B, int Hq, int Hkv, int Tq,
+                       int Tk, int cached, int d, int window, float scale,
+                       int32_t *dev_status, gqa_stream_t stream) {
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
   if (B < 0 || Tq < 0 || Tk < 0) return GQA_ERR_SHAPE;
   gqa_status s = check_heads(Hq, Hkv, d);
@@ -319,6 +320,7 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
   if (B == 0 || Tq == 0) return GQA_OK;
   if (!q || !k || !v || !o) return GQA_ERR_NULL;
   if (cached && (!seq_lens || !dev_status)) return GQA_ERR_NULL;
+  if (seg && !dev_status) return GQA_ERR_NULL;
   if (d > GQA_MAX_HEAD_DIM) return GQA_ERR_UNSUPPORTED;
   DeviceInfo di;
   if ((s = device_info(&di)) != GQA_OK) return s;
@@ -329,16 +331,17 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
     // Heads of a group in pairs (one CTA per pair) when the group size is
     // even; otherwise one head per CTA.
     if (gqa::pf2::supported(d, Hq, Hkv))
-      return gqa::pf2::launch(q, k, v, o, seq_lens, B, Hq, Hkv, Tq, Tk, cached, d,
-                              window, scale_log2, dev_status, st);
-    return gqa::pf::launch(q, k, v, o, seq_lens, B, Hq, Hkv, Tq, Tk, cached, d,
+      return gqa::pf2::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached,
+                              d, window, scale_log2, dev_status, st);
+    return gqa::pf::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,
                            window, scale_log2, dev_status, st);
   }
   if (Hq > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
   if (dtype == GQA_F32)
-    return launch_simt_prefill<float>(q, k, v, o, seq_lens, B, Hq, Hkv, Tq, Tk,
-                                      cached, d, window, scale_log2, dev_status, st);
-  return launch_simt_prefill<bf16>(q, k, v, o, seq_lens, B, Hq, Hkv, Tq, Tk,
+    return launch_simt_prefill<float>(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq,
+                                      Tk, cached, d, window, scale_log2,
+                                      dev_status, st);
+  return launch_simt_prefill<bf16>(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk,
                                    cached, d, window, scale_log2, dev_status, st);
 }
 
@@ -350,8 +353,18 @@ gqa_status gqa_prefill(gqa_dtype dtype, const void *q, const void *k,
                        const void *v, void *o, const int32_t *seq_lens, int B,
                        int Hq, int Hkv, int T, int d, int window, float scale,
                        int32_t *dev_status, gqa_stream_t stream) {
-  return attend_impl(dtype, q, k, v, o, seq_lens, B, Hq, Hkv, T, T, 0, d, window,
-                     scale, dev_status, stream);
+  return attend_impl(dtype, q, k, v, o, seq_lens, nullptr, B, Hq, Hkv, T, T, 0, d,
+                     window, scale, dev_status, stream);
+}
+
+gqa_status gqa_prefill_packed(gqa_dtype dtype, const void *q, const void *k,
+                              const void *v, void *o, const int32_t *seq_lens,
+                              const int32_t *seg_start, int B, int Hq, int Hkv,
+                              int T, int d, int window, float scale,
+                              int32_t *dev_status, gqa_stream_t stream) {
+  if (B > 0 && T > 0 && !seg_start) return GQA_ERR_NULL;
+  return attend_impl(dtype, q, k, v, o, seq_lens, seg_start, B, Hq, Hkv, T, T, 0, d,
+                     window, scale, dev_status, stream);
 }
 
 gqa_status gqa_decode_multi(gqa_dtype dtype, const void *q, const void *k_cache,
@@ -361,8 +374,8 @@ gqa_status gqa_decode_multi(gqa_dtype dtype, const void *q, const void *k_cache,
                             gqa_stream_t stream) {
   if (C < 0 || t_new < 0) return GQA_ERR_SHAPE;
   if (t_new > C) return GQA_ERR_CAPACITY;
-  return attend_impl(dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, t_new, C,
-                     1, d, window, scale, dev_status, stream);
+  return attend_impl(dtype, q, k_cache, v_cache, o, seq_lens, nullptr, B, Hq, Hkv,
+                     t_new, C, 1, d, window, scale, dev_status, stream);
 }
 
 size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,

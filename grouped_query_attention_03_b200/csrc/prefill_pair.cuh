@@ -69,8 +69,22 @@ struct Params {
   int Tk;      // key rows per KV lane (K and V are [B,Hkv,Tk,d])
   int cached;  // 0: prompt, query row t at position t, n_b = active rows;
                // 1: queries after a cache, query row i at position n_b-Tq+i
+  const int32_t *seg;  // prompt only: [B,Tq] first key cell of row t's
+                       // packed segment, or NULL (segment start 0)
   float scale_log2;
 };
+
+// First permitted key of query position t ("Intersect the window with the
+// context already permitted": the later of the segment start and the
+// window start); t + 1 (no key) when the segment start is not in [0, t].
+__device__ __forceinline__ int row_lo(const Params &p, int b, int t) {
+  int s0 = 0;
+  if (p.seg) {
+    s0 = p.seg[(size_t)b * p.Tq + t];
+    if (s0 < 0 || s0 > t) return t + 1;
+  }
+  return p.window > 0 ? max(s0, t - (p.window - 1)) : s0;
+}
 
 struct Bars {
   uint64_t q_full;
@@ -128,8 +142,8 @@ __device__ __forceinline__ float emit_p(const float *s, float sc, float m, unsig
 template <int D>
 __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsigned char *smem,
                                              uint32_t tmem, int hd, int b, int h, int m0,
-                                             int a0, int a_end, int n_keys, int j0, int nt,
-                                             bool *failed) {
+                                             int a0, int a_end, int n_keys, int lo_max, int j0,
+                                             int nt, bool *failed) {
   using K = Cfg<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3;
@@ -137,7 +151,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
   const int t = a0 + row;       // key position of this query row
   const int qr = m0 + row;      // its row in Q and O
   const bool active = t < a_end;
-  const int lo_t = p.window > 0 ? max(0, t - (p.window - 1)) : 0;
+  const int lo_t = active ? row_lo(p, b, t) : 0;
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
   const uint32_t tS = tmem + lane_base + hd * kBN;
   const uint32_t tO = tmem + lane_base + K::TM_O + hd * D;
@@ -149,7 +163,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
     const int kb = (j0 + j) * kBN;
     if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[hd], j & 1, failed))) { ok = false; break; }
     tc::fence_after_sync();
-    const bool edge = (kb + kBN - 1 > a0) || (p.window > 0 && kb < a0 + kBM - p.window);
+    const bool edge = (kb + kBN - 1 > a0) || (kb < lo_max);
     // the whole row of scores: four TMEM loads, one wait
     float s[kBN];
 #pragma unroll
@@ -290,12 +304,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int off = (p.cached && n_b >= 0) ? n_b - p.Tq : 0;
   const int rows = n_b < 0 ? 0 : (p.cached ? p.Tq : n_b);
   const int a0 = off + m0;
-  int j0 = 0, nt = 0;
-  if (rows > m0) {
-    const int lo = p.window > 0 ? max(0, a0 - (p.window - 1)) : 0;
-    const int hi = min(a0 + kBM - 1, off + rows - 1);
-    j0 = lo / kBN;
-    nt = hi / kBN - j0 + 1;
+  // Packed segments: the tile's rows (one per thread of warps 0-3) give the
+  // smallest and largest first permitted key; invalid starts are reported.
+  __shared__ int s_lo_min[4], s_lo_max[4];
+  if (p.seg && warp < 4) {
+    const int t = a0 + (int)threadIdx.x;
+    int lmin = 0x7fffffff, lmax = -1;
+    if (t < off + rows) {
+      const int lo = row_lo(p, b, t);
+      if (lo > t) {
+        record_status(p.status, GQA_ERR_SEGMENT);
+      } else {
+        lmin = lo;
+        lmax = lo;
+      }
+    }
+    lmin = __reduce_min_sync(0xffffffffu, lmin);
+    lmax = __reduce_max_sync(0xffffffffu, lmax);
+    if (lane == 0) {
+      s_lo_min[warp] = lmin;
+      s_lo_max[warp] = lmax;
+    }
   }
 
   if (threadIdx.x == 0) {
@@ -319,14 +348,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
+  // KV tiles [j0, j0 + nt) cover the tile's permitted keys; tiles starting
+  // before lo_max need masks (some row's first key lies inside them).
+  int lo_min, lo_max;
+  if (p.seg) {
+    lo_min = min(min(s_lo_min[0], s_lo_min[1]), min(s_lo_min[2], s_lo_min[3]));
+    lo_max = max(max(s_lo_max[0], s_lo_max[1]), max(s_lo_max[2], s_lo_max[3]));
+  } else {
+    lo_min = p.window > 0 ? max(0, a0 - (p.window - 1)) : 0;
+    lo_max = p.window > 0 ? max(0, a0 + kBM - p.window) : 0;
+  }
+  int j0 = 0, nt = 0;
+  if (rows > m0 && lo_min != 0x7fffffff) {
+    const int hi = min(a0 + kBM - 1, off + rows - 1);
+    j0 = lo_min / kBN;
+    nt = hi / kBN - j0 + 1;
+  }
   const uint32_t tmem = bars.tmem_base;
   bool failed = false;
   if (warp >= 4) {
     // ================================================= softmax warpgroups
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     const int hd = (warp - 4) / 4;  // warps 4-7: head A, 8-11: head B
-    softmax_head<D>(p, bars, smem, tmem, hd, b, h0 + hd, m0, a0, off + rows, max(n_b, 0), j0,
-                    nt, &failed);
+    softmax_head<D>(p, bars, smem, tmem, hd, b, h0 + hd, m0, a0, off + rows, max(n_b, 0),
+                    lo_max, j0, nt, &failed);
   } else {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
@@ -445,9 +490,9 @@ inline bool supported(int d, int Hq, int Hkv) {
 
 template <int D>
 gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
-                    const int32_t *lens, int B, int Hq, int Hkv, int Tq, int Tk,
-                    int cached, int window, float scale_log2, int32_t *status,
-                    cudaStream_t st) {
+                    const int32_t *lens, const int32_t *seg, int B, int Hq, int Hkv,
+                    int Tq, int Tk, int cached, int window, float scale_log2,
+                    int32_t *status, cudaStream_t st) {
   using K = Cfg<D>;
   CUtensorMap mq, mk, mv;
   if (!tma::make_bf16_map(&mq, q, D, Tq, B * Hq, 128) ||
@@ -474,6 +519,7 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.Tq = Tq;
   p.Tk = Tk;
   p.cached = cached;
+  p.seg = seg;
   p.window = window;
   p.num_mt = (Tq + kBM - 1) / kBM;
   p.pairs = (Hq / Hkv) / 2;
@@ -487,14 +533,14 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
 // Prompt (cached = 0: Tq = Tk = T) or queries after a cache (cached = 1:
 // Tq new rows against Tk = capacity cells).
 inline gqa_status launch(const void *q, const void *k, const void *v, void *o,
-                         const int32_t *lens, int B, int Hq, int Hkv, int Tq, int Tk,
-                         int cached, int d, int window, float scale_log2, int32_t *status,
-                         cudaStream_t st) {
+                         const int32_t *lens, const int32_t *seg, int B, int Hq, int Hkv,
+                         int Tq, int Tk, int cached, int d, int window, float scale_log2,
+                         int32_t *status, cudaStream_t st) {
   if (d == 64)
-    return launch_d<64>(q, k, v, o, lens, B, Hq, Hkv, Tq, Tk, cached, window, scale_log2,
-                        status, st);
-  return launch_d<128>(q, k, v, o, lens, B, Hq, Hkv, Tq, Tk, cached, window, scale_log2,
-                       status, st);
+    return launch_d<64>(q, k, v, o, lens, seg, B, Hq, Hkv, Tq, Tk, cached, window,
+                        scale_log2, status, st);
+  return launch_d<128>(q, k, v, o, lens, seg, B, Hq, Hkv, Tq, Tk, cached, window,
+                       scale_log2, status, st);
 }
 
 }  // namespace pf2

@@ -94,14 +94,16 @@ __device__ void zero_row_warp(T *orow, int d) {
 // are [B,Hq,Tq,d], K and V [B,Hkv,Tk,d].  cached = 0: a prompt (Tq = Tk),
 // row i at key position i, rows i >= n_b zero.  cached = 1: Tq new rows
 // after a cache of n_b cells (the new ones included), row i at position
-// n_b - Tq + i.
+// n_b - Tq + i.  seg (prompt only, or NULL): [B,Tq] first key cell of
+// row t's packed segment; a start outside [0, t] gives a zero row and
+// GQA_ERR_SEGMENT.
 template <typename T, int NF>
 __global__ void __launch_bounds__(128)
     prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
                         const T *__restrict__ v, T *__restrict__ o,
-                        const int32_t *__restrict__ seq_lens, int Hq, int Hkv,
-                        int Tq, int Tk, int cached, int d, int window,
-                        float scale_log2, int32_t *status) {
+                        const int32_t *__restrict__ seq_lens, const int32_t *seg,
+                        int Hq, int Hkv, int Tq, int Tk, int cached, int d,
+                        int window, float scale_log2, int32_t *status) {
   const int i = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int h = blockIdx.y, b = blockIdx.z;
   if (i >= Tq) return;
@@ -122,7 +124,16 @@ __global__ void __launch_bounds__(128)
     zero_row_warp<T, NF>(orow, d);
     return;
   }
-  const int lo = window > 0 ? max(0, t - (window - 1)) : 0;
+  int s0 = 0;
+  if (seg) {
+    s0 = seg[(size_t)b * Tq + t];
+    if (s0 < 0 || s0 > t) {
+      if ((threadIdx.x & 31) == 0) record_status(status, GQA_ERR_SEGMENT);
+      zero_row_warp<T, NF>(orow, d);
+      return;
+    }
+  }
+  const int lo = window > 0 ? max(s0, t - (window - 1)) : s0;
   const size_t lane_off = ((size_t)b * Hkv + g) * Tk * d;
   attend_row_warp<T, NF>(q + (((size_t)b * Hq + h) * Tq + i) * d,
                          k + lane_off, v + lane_off, lo, t, d, scale_log2,

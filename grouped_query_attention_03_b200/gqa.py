@@ -22,11 +22,11 @@ STATUS_NAMES = {
     0: "GQA_OK", 1: "GQA_ERR_NULL", 2: "GQA_ERR_SHAPE", 3: "GQA_ERR_GROUPS",
     4: "GQA_ERR_WINDOW", 5: "GQA_ERR_CAPACITY", 6: "GQA_ERR_OVERFLOW",
     7: "GQA_ERR_UNSUPPORTED", 8: "GQA_ERR_WORKSPACE", 9: "GQA_ERR_CUDA",
-    10: "GQA_ERR_DEVICE", 11: "GQA_ERR_TIMEOUT",
+    10: "GQA_ERR_DEVICE", 11: "GQA_ERR_TIMEOUT", 12: "GQA_ERR_SEGMENT",
 }
 
 # Every symbol include/gqa.h declares.
-EXPORTS = ("gqa_prefill", "gqa_decode", "gqa_decode_workspace_bytes",
+EXPORTS = ("gqa_prefill", "gqa_prefill_packed", "gqa_decode", "gqa_decode_workspace_bytes",
            "gqa_decode_append", "gqa_decode_multi", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
            "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
            "gqa_version")
@@ -61,6 +61,8 @@ def _declare(L):
     sz, i64 = ctypes.c_size_t, ctypes.c_int64
     L.gqa_prefill.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, vp]
     L.gqa_prefill.restype = i32
+    L.gqa_prefill_packed.argtypes = [i32, vp, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, vp]
+    L.gqa_prefill_packed.restype = i32
     L.gqa_decode.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 6 + [f32, vp, sz, vp, vp]
     L.gqa_decode.restype = i32
     L.gqa_decode_append.argtypes = [i32] + [vp] * 7 + [i32] * 6 + [f32, vp, sz, vp, vp]
@@ -154,6 +156,31 @@ def prefill(q, k, v, *, window=None, scale=None, seq_lens=None, out=None,
         _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
         B, Hq, Hkv, T, d, _window(window), float(scale),
         _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_prefill")
+    return out
+
+
+def prefill_packed(q, k, v, seg_start, *, window=None, scale=None, seq_lens=None,
+                   out=None, status=None, stream=None):
+    """prefill() over packed sequences: seg_start [B,T] int32 holds each
+    cell's segment start; cell t attends [max(seg_start, t-(w-1)), t]."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    if tuple(seg_start.shape) != (B, T):
+        raise ValueError("seg_start must be [B, T]")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_prefill_packed(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k, "k", q.dtype, dev), _ptr(v, "v", q.dtype, dev),
+        _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
+        _ptr(seg_start, "seg_start", torch.int32, dev),
+        B, Hq, Hkv, T, d, _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
+        _stream(stream, dev)), "gqa_prefill_packed")
     return out
 
 

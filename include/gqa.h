@@ -68,8 +68,10 @@ typedef enum {
   GQA_ERR_WORKSPACE = 8,   /* workspace NULL or smaller than required */
   GQA_ERR_CUDA = 9,        /* a CUDA runtime call or launch failed */
   GQA_ERR_DEVICE = 10,     /* the current device is not sm_100 */
-  GQA_ERR_TIMEOUT = 11     /* a kernel's bounded internal wait ran out (set
+  GQA_ERR_TIMEOUT = 11,    /* a kernel's bounded internal wait ran out (set
                               in *dev_status only) */
+  GQA_ERR_SEGMENT = 12     /* a packed segment start s_{b,t} lies outside
+                              [0, t] (set in *dev_status only) */
 } gqa_status;
 
 #define GQA_NO_WINDOW (-1)
@@ -99,6 +101,26 @@ gqa_status gqa_prefill(gqa_dtype dtype, const void *q, const void *k,
                        const void *v, void *o, const int32_t *seq_lens,
                        int B, int Hq, int Hkv, int T, int d, int window,
                        float scale, int32_t *dev_status, gqa_stream_t stream);
+
+/*
+ * gqa_prefill_packed -- gqa_prefill over packed sequences: several
+ * documents share one row of the batch, and a query sees only its own
+ * document.  [P1] "Intersect the window with the context already
+ * permitted": the first permitted key of cell t is the later of its
+ * segment start s_{b,t} and the window start t - (w-1) (saturating), so
+ * cell t reads keys [max(s_{b,t}, t-(w-1)), t].
+ *
+ *   seg_start device int32 [B,T]: s_{b,t}, the first cell of t's segment
+ *            (required; only cells t < n_b are read)
+ *   everything else as for gqa_prefill.
+ * A start outside [0, t] gives that query row no keys: its output is zero
+ * and *dev_status is set to GQA_ERR_SEGMENT (dev_status is required).
+ */
+gqa_status gqa_prefill_packed(gqa_dtype dtype, const void *q, const void *k,
+                              const void *v, void *o, const int32_t *seq_lens,
+                              const int32_t *seg_start, int B, int Hq, int Hkv,
+                              int T, int d, int window, float scale,
+                              int32_t *dev_status, gqa_stream_t stream);
 
 /*
  * gqa_decode -- one new query token per sequence against the KV cache.

@@ -45,8 +45,9 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_version_and_strings(L):
     assert L.gqa_version().decode().count(".") == 2
-    for code in range(12):
+    for code in range(13):
         assert L.gqa_status_string(code)
+        assert L.gqa_status_string(code) != b"unknown status"
     assert L.gqa_status_string(999) == b"unknown status"
 
 
@@ -130,6 +131,24 @@ def test_decode_multi_host_refusals(L):
     assert _decode_multi(L, q=None) == NULL
     assert _decode_multi(L, t_new=0, q=None) == OK
     assert _decode_multi(L, B=0, q=None) == OK
+
+
+def test_prefill_packed_host_refusals(L):
+    f = L.gqa_prefill_packed
+    args = [1, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 4, 2, 8, 64, -1, 0.125, FAKE, None]
+    bad_seg = list(args)
+    bad_seg[6] = None
+    assert f(*bad_seg) == NULL
+    no_status = list(args)
+    no_status[14] = None
+    assert f(*no_status) == NULL
+    groups = list(args)
+    groups[8] = 3
+    assert f(*groups) == GROUPS
+    empty = list(args)
+    empty[7] = 0
+    empty[6] = None
+    assert f(*empty) == OK
 
 
 def test_prefill_host_refusals(L):
