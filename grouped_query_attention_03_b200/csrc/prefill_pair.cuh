@@ -77,9 +77,10 @@ struct Params {
 // First permitted key of query position t ("Intersect the window with the
 // context already permitted": the later of the segment start and the
 // window start); t + 1 (no key) when the segment start is not in [0, t].
+template <bool SEG>
 __device__ __forceinline__ int row_lo(const Params &p, int b, int t) {
   int s0 = 0;
-  if (p.seg) {
+  if (SEG) {
     s0 = p.seg[(size_t)b * p.Tq + t];
     if (s0 < 0 || s0 > t) return t + 1;
   }
@@ -91,6 +92,7 @@ struct Bars {
   uint64_t full[6], empty[6];
   uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t mma_fin;
+  uint64_t v_clean;  // the last V tile's rows past the sequence are zero
   uint32_t tmem_base;
 };
 
@@ -139,11 +141,11 @@ __device__ __forceinline__ float emit_p(const float *s, float sc, float m, unsig
 
 // Softmax and epilogue for one head (one 128-thread warpgroup, TMEM lanes
 // = query rows).  `hd` selects the head's S/O columns, P buffer, barriers.
-template <int D>
+template <int D, bool SEG>
 __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsigned char *smem,
                                              uint32_t tmem, int hd, int b, int h, int m0,
-                                             int a0, int a_end, int n_keys, int lo_max, int j0,
-                                             int nt, bool *failed) {
+                                             int a0, int a_end, int lo_max, int j0, int nt,
+                                             bool *failed) {
   using K = Cfg<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q4 = warp & 3;
@@ -151,7 +153,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
   const int t = a0 + row;       // key position of this query row
   const int qr = m0 + row;      // its row in Q and O
   const bool active = t < a_end;
-  const int lo_t = active ? row_lo(p, b, t) : 0;
+  const int lo_t = active ? row_lo<SEG>(p, b, t) : 0;
   const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
   const uint32_t tS = tmem + lane_base + hd * kBN;
   const uint32_t tO = tmem + lane_base + K::TM_O + hd * D;
@@ -210,26 +212,6 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
       m_run = m_new;
     }
     const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, sP, row);
-    if (hd == 0 && kb + kBN > n_keys) {
-      // Cells past the sequence in this V tile are not the sequence's (an
-      // unwritten cache cell may hold NaN): their p is 0, but 0 * NaN is not,
-      // so head A's threads clear those rows (thread = row) before either
-      // head's P V is issued (head B's comes after head A's).
-      const int i = 2 * j + 1;  // the producer's fill index of V_j
-      const int slot = i % K::NSLOT;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.full[slot], (i / K::NSLOT) & 1, failed))) {
-        ok = false;
-        break;
-      }
-      if (kb + row >= n_keys) {
-        unsigned char *vrow = smem + K::OFF_RING + slot * K::TILE + row * 128;
-#pragma unroll
-        for (int c = 0; c < K::KB; ++c)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4 *>(vrow + c * K::BLK + ch * 16) = make_uint4(0, 0, 0, 0);
-      }
-    }
     l_run += lsum;
     tc::fence_proxy_async_smem();
     tc::fence_before_sync();
@@ -269,7 +251,9 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
   }
 }
 
-template <int D>
+// SEG: packed segment starts are given (p.seg); the plain prompt and the
+// cached-query forms compile without that code.
+template <int D, bool SEG>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -307,11 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Packed segments: the tile's rows (one per thread of warps 0-3) give the
   // smallest and largest first permitted key; invalid starts are reported.
   __shared__ int s_lo_min[4], s_lo_max[4];
-  if (p.seg && warp < 4) {
+  if (SEG && warp < 4) {
     const int t = a0 + (int)threadIdx.x;
     int lmin = 0x7fffffff, lmax = -1;
     if (t < off + rows) {
-      const int lo = row_lo(p, b, t);
+      const int lo = row_lo<SEG>(p, b, t);
       if (lo > t) {
         record_status(p.status, GQA_ERR_SEGMENT);
       } else {
@@ -339,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.o_done[h], 1);
     }
     mbar_init(&bars.mma_fin, 1);
+    mbar_init(&bars.v_clean, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -351,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // KV tiles [j0, j0 + nt) cover the tile's permitted keys; tiles starting
   // before lo_max need masks (some row's first key lies inside them).
   int lo_min, lo_max;
-  if (p.seg) {
+  if (SEG) {
     lo_min = min(min(s_lo_min[0], s_lo_min[1]), min(s_lo_min[2], s_lo_min[3]));
     lo_max = max(max(s_lo_max[0], s_lo_max[1]), max(s_lo_max[2], s_lo_max[3]));
   } else {
@@ -364,14 +349,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     j0 = lo_min / kBN;
     nt = hi / kBN - j0 + 1;
   }
+  // Rows [z0, z1) of the last V tile are cells past the sequence that exist
+  // in memory (an unwritten cache cell or prompt padding may hold NaN):
+  // their p is 0, but 0 * NaN is not, so they are cleared before P V.
+  const int kb_last = (j0 + nt - 1) * kBN;
+  const int z0 = max(0, max(n_b, 0) - kb_last), z1 = min(kBN, p.Tk - kb_last);
+  const bool clear_v = nt > 0 && z0 < z1;
   const uint32_t tmem = bars.tmem_base;
   bool failed = false;
   if (warp >= 4) {
     // ================================================= softmax warpgroups
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     const int hd = (warp - 4) / 4;  // warps 4-7: head A, 8-11: head B
-    softmax_head<D>(p, bars, smem, tmem, hd, b, h0 + hd, m0, a0, off + rows, max(n_b, 0),
-                    lo_max, j0, nt, &failed);
+    softmax_head<D, SEG>(p, bars, smem, tmem, hd, b, h0 + hd, m0, a0, off + rows, lo_max, j0,
+                         nt, &failed);
   } else {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
@@ -408,6 +399,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < K::NSLOT; ++s)
         if (fills[s] > 0) mbar_wait(&bars.full[s], (fills[s] - 1) & 1, &f2);
       failed |= f2;
+    }
+    if (clear_v) {
+      // every copy has landed (lane 0 waited above): clear, then release
+      __syncwarp();
+      unsigned char *vt = smem + K::OFF_RING + ((2 * nt - 1) % K::NSLOT) * K::TILE;
+      for (int idx = lane; idx < (z1 - z0) * K::KB * 8; idx += 32) {
+        const int r = z0 + idx / (K::KB * 8), c = (idx / 8) % K::KB, ch = idx % 8;
+        *reinterpret_cast<uint4 *>(vt + c * K::BLK + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+      }
+      tc::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.v_clean);
     }
   } else if (warp == 1) {
     // ================================================= MMA issuer
@@ -450,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nt; ++j) {
         // head A: O_A += P_A(j) V_j, then S_A(j+1)
         if (!mbar_wait(&bars.p_full[0], j & 1, &failed) || !wait_load(2 * j + 1)) { ok = false; break; }
+        if (clear_v && j == nt - 1 && !mbar_wait(&bars.v_clean, 0, &failed)) { ok = false; break; }
         tc::fence_after_sync();
         issue_pv(0, j);
         if (j + 1 < nt) {
@@ -499,9 +503,12 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
       !tma::make_bf16_map(&mk, k, D, Tk, B * Hkv, 128) ||
       !tma::make_bf16_map(&mv, v, D, Tk, B * Hkv, 128))
     return GQA_ERR_CUDA;
-  static bool attr_done = false;
+  static bool attr_done = false;  // per instantiation; benign race
   if (!attr_done) {
-    if (cudaFuncSetAttribute(prefill_pair_kernel<D>,
+    if (cudaFuncSetAttribute(prefill_pair_kernel<D, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             K::SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(prefill_pair_kernel<D, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              K::SMEM) != cudaSuccess) {
       cudaGetLastError();
@@ -526,7 +533,10 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.scale_log2 = scale_log2;
   const long long grid = (long long)B * Hkv * p.pairs * p.num_mt;
   if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
-  prefill_pair_kernel<D><<<(unsigned)grid, kThreads, K::SMEM, st>>>(mq, mk, mv, p);
+  if (seg)
+    prefill_pair_kernel<D, true><<<(unsigned)grid, kThreads, K::SMEM, st>>>(mq, mk, mv, p);
+  else
+    prefill_pair_kernel<D, false><<<(unsigned)grid, kThreads, K::SMEM, st>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
