@@ -53,6 +53,10 @@ def _load(path):
     L.oracle_decode_multi.restype = ctypes.c_int
     L.oracle_cache_append.argtypes = [dp, dp, dp, dp, lp] + [c_long] * 5
     L.oracle_cache_append.restype = ctypes.c_int
+    L.oracle_ring_append.argtypes = [dp, dp, dp, dp, lp] + [c_long] * 5
+    L.oracle_ring_append.restype = ctypes.c_int
+    L.oracle_ring_decode.argtypes = [dp, dp, dp, dp, lp] + [c_long] * 5 + [c_double]
+    L.oracle_ring_decode.restype = ctypes.c_int
     L.oracle_cache_bytes.argtypes = [ctypes.c_uint64] * 6
     L.oracle_cache_bytes.restype = ctypes.c_uint64
     L.oracle_set_threads.argtypes = [ctypes.c_int]
@@ -176,6 +180,36 @@ def cache_append(k_cache, v_cache, k_new, v_new, seq_lens):
                                    B, Hkv, C, d, t_new)
     _check(rc, "cache_append")
     return kc, vc, lens
+
+
+def ring_append(k_ring, v_ring, k_new, v_new, seq_lens):
+    """Rolling buffer of W slots: writes positions [len_b, len_b + t_new) at
+    slots p mod W (the last W survive).  Returns (k_ring', v_ring',
+    seq_lens') as new arrays, or raises OracleError."""
+    kr, vr = _f64(k_ring).copy(), _f64(v_ring).copy()
+    kn, vn = _f64(k_new), _f64(v_new)
+    lens = _lens(seq_lens).copy()
+    B, Hkv, W, d = kr.shape
+    t_new = kn.shape[2]
+    rc = lib().oracle_ring_append(_dp(kr), _dp(vr), _dp(kn), _dp(vn), _lp(lens),
+                                  B, Hkv, W, d, t_new)
+    _check(rc, "ring_append")
+    return kr, vr, lens
+
+
+def ring_decode(q, k_ring, v_ring, seq_lens, scale=None):
+    """Decode against a rolling buffer: the query at position n_b - 1 reads
+    positions [max(0, n_b - W), n_b) from their slots.  q [B,Hq,d]."""
+    q, kr, vr = _f64(q), _f64(k_ring), _f64(v_ring)
+    B, Hq, d = q.shape
+    Hkv, W = kr.shape[1], kr.shape[2]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.empty((B, Hq, d), dtype=np.float64)
+    rc = lib().oracle_ring_decode(_dp(q), _dp(kr), _dp(vr), _dp(o), _lp(_lens(seq_lens)),
+                                  B, Hq, Hkv, W, d, float(scale))
+    _check(rc, "ring_decode")
+    return o
 
 
 def cache_bytes(L, B, T, Hkv, d, e):

@@ -231,6 +231,76 @@ int oracle_cache_append(double *k_cache, double *v_cache, const double *k_new,
   return 0;
 }
 
+/* Rolling buffer: position p in slot p mod W ([P1] "Relate shared heads to
+ * local context"). */
+int oracle_ring_append(double *k_ring, double *v_ring, const double *k_new,
+                       const double *v_new, long *seq_lens, long B, long Hkv,
+                       long W, long d, long t_new) {
+  if (B < 0 || W <= 0 || t_new < 0 || Hkv <= 0 || d <= 0) return 1;
+  if (B == 0 || t_new == 0) return 0;
+  if (!k_ring || !v_ring || !k_new || !v_new || !seq_lens) return 1;
+  for (long b = 0; b < B; ++b)
+    if (seq_lens[b] < 0 || seq_lens[b] > 2147483647L - t_new) return 2;
+  for (long b = 0; b < B; ++b) {
+    for (long g = 0; g < Hkv; ++g)
+      for (long i = 0; i < t_new; ++i) {
+        long pos = seq_lens[b] + i;
+        if (t_new - i > W) continue; /* overwritten by a later new row */
+        long dst = ((b * Hkv + g) * W + pos % W) * d;
+        long src = ((b * Hkv + g) * t_new + i) * d;
+        memcpy(k_ring + dst, k_new + src, sizeof(double) * (size_t)d);
+        memcpy(v_ring + dst, v_new + src, sizeof(double) * (size_t)d);
+      }
+    seq_lens[b] += t_new;
+  }
+  return 0;
+}
+
+int oracle_ring_decode(const double *q, const double *k_ring,
+                       const double *v_ring, double *o, const long *seq_lens,
+                       long B, long Hq, long Hkv, long W, long d, double scale) {
+  if (B < 0 || W <= 0 || check_heads(Hq, Hkv, d)) return 1;
+  if (B == 0) return 0;
+  if (!q || !k_ring || !v_ring || !o || !seq_lens) return 1;
+  for (long b = 0; b < B; ++b)
+    if (seq_lens[b] < 0) return 2;
+  long r = Hq / Hkv;
+  int bad = 0;
+#pragma omp parallel num_threads(g_threads) reduction(| : bad)
+  {
+    /* the window's keys and values gathered in position order */
+    double *kk = (double *)malloc(sizeof(double) * (size_t)(W * d));
+    double *vv = (double *)malloc(sizeof(double) * (size_t)(W * d));
+    double *scratch = (double *)malloc(sizeof(double) * (size_t)W);
+    if (!kk || !vv || !scratch) bad = 1;
+#pragma omp for collapse(2) schedule(dynamic)
+    for (long b = 0; b < B; ++b) {
+      for (long h = 0; h < Hq; ++h) {
+        if (!kk || !vv || !scratch) continue;
+        long n = seq_lens[b];
+        double *orow = o + (b * Hq + h) * d;
+        if (n == 0) {
+          memset(orow, 0, sizeof(double) * (size_t)d);
+          continue;
+        }
+        long g = h / r;
+        long lo = n > W ? n - W : 0;
+        for (long pos = lo; pos < n; ++pos) {
+          long src = ((b * Hkv + g) * W + pos % W) * d;
+          memcpy(kk + (pos - lo) * d, k_ring + src, sizeof(double) * (size_t)d);
+          memcpy(vv + (pos - lo) * d, v_ring + src, sizeof(double) * (size_t)d);
+        }
+        attend_row(q + (b * Hq + h) * d, kk, vv, 0, n - 1 - lo, d, scale, orow,
+                   NULL, scratch);
+      }
+    }
+    free(kk);
+    free(vv);
+    free(scratch);
+  }
+  return bad ? 1 : 0;
+}
+
 /* [P3] M_KV = 2 L B T Hkv d e, checked for uint64 overflow. */
 uint64_t oracle_cache_bytes(uint64_t L, uint64_t B, uint64_t T, uint64_t Hkv,
                             uint64_t d, uint64_t e) {

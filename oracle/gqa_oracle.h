@@ -72,6 +72,24 @@ int oracle_cache_append(double *k_cache, double *v_cache, const double *k_new,
                         const double *v_new, long *seq_lens, long B, long Hkv,
                         long C, long d, long t_new);
 
+/* Rolling-buffer (ring) cache of W slots per lane ([P1] "Relate shared heads
+ * to local context": a rolling buffer that overwrites old KV entries; the
+ * chapter does not implement it).  Reading: position p lives in slot
+ * p mod W.  Append writes positions [len_b, len_b + t_new) (only the last W
+ * of them survive) and advances seq_lens; refused (nothing written) if a
+ * length is negative or would overflow. */
+int oracle_ring_append(double *k_ring, double *v_ring, const double *k_new,
+                       const double *v_new, long *seq_lens, long B, long Hkv,
+                       long W, long d, long t_new);
+
+/* Decode against a ring: n_b = seq_lens[b] positions so far (the current
+ * token included); the query at position n_b - 1 reads positions
+ * [max(0, n_b - W), n_b) from their slots, in position order (a window of W
+ * cells over the positions). */
+int oracle_ring_decode(const double *q, const double *k_ring,
+                       const double *v_ring, double *o, const long *seq_lens,
+                       long B, long Hq, long Hkv, long W, long d, double scale);
+
 /* [P3] "Computing the cache requirement": 2*L*B*T*Hkv*d*e, 0 on overflow. */
 uint64_t oracle_cache_bytes(uint64_t L, uint64_t B, uint64_t T, uint64_t Hkv,
                             uint64_t d, uint64_t e);

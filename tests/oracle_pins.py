@@ -319,6 +319,63 @@ def pin_cache_append(O):
         raise AssertionError("append beyond capacity was accepted")
 
 
+def pin_ring_equals_windowed_decode(O):
+    """A rolling buffer of W slots ("Relate shared heads to local context":
+    Mistral's rolling buffer that overwrites old KV entries; the chapter does
+    not build it) holds exactly the last W positions, so decoding against it
+    equals decoding with window W against the all-prefix cache that the
+    chapter keeps -- bit for bit, since both read the same keys in position
+    order.  Appends come in random chunk sizes, some longer than W."""
+    r = _rng(21)
+    B, Hq, Hkv, d = 2, 4, 2, 3
+    for W in (1, 2, 3, 5, 8):
+        kr = np.zeros((B, Hkv, W, d))
+        vr = np.zeros((B, Hkv, W, d))
+        C = 40
+        kc = np.zeros((B, Hkv, C, d))
+        vc = np.zeros((B, Hkv, C, d))
+        lr = np.zeros(B, dtype=np.int64)
+        lc = np.zeros(B, dtype=np.int64)
+        while lc.max() < 30:
+            t_new = int(r.integers(1, 2 * W + 2))
+            if lc.max() + t_new > C:
+                break
+            kn = r.standard_normal((B, Hkv, t_new, d))
+            vn = r.standard_normal((B, Hkv, t_new, d))
+            kr, vr, lr = O.ring_append(kr, vr, kn, vn, lr)
+            kc, vc, lc = O.cache_append(kc, vc, kn, vn, lc)
+            assert lr.tolist() == lc.tolist()
+            # every surviving slot holds the row of its position
+            for b in range(B):
+                n = lc[b]
+                for pos in range(max(0, n - W), n):
+                    assert np.array_equal(kr[b, :, pos % W], kc[b, :, pos])
+                    assert np.array_equal(vr[b, :, pos % W], vc[b, :, pos])
+            q = r.standard_normal((B, Hq, d))
+            want = O.decode(q, kc, vc, lc, window=W)
+            got = O.ring_decode(q, kr, vr, lr)
+            assert np.array_equal(got, want), W
+
+
+def pin_ring_refusals(O):
+    """Negative lengths and an empty ring are refused."""
+    kr = np.zeros((1, 1, 4, 2))
+    one = np.zeros((1, 1, 1, 2))
+    for lens, ring in (([-1], kr), ([0], np.zeros((1, 1, 0, 2)))):
+        try:
+            O.ring_append(ring, ring, one, one, lens)
+        except O.OracleError:
+            pass
+        else:
+            raise AssertionError(f"ring append accepted {lens}, W={ring.shape[2]}")
+    try:
+        O.ring_decode(np.zeros((1, 2, 2)), kr, kr, [-2])
+    except O.OracleError:
+        pass
+    else:
+        raise AssertionError("ring decode accepted a negative length")
+
+
 def pin_refusals(O):
     """Zero window refused; indivisible heads refused."""
     q = np.zeros((1, 3, 2, 2))

@@ -37,6 +37,10 @@ MUTATIONS = [
     ("bytes_factor", "uint64_t acc = 2;", "uint64_t acc = 1;"),
     ("segment_ignored", "long s0 = seg_start ? seg_start[b * T + t] : 0;", "long s0 = 0;"),
     ("query_row_index", "attend_row(q + ((b * Hq + h) * T + t) * d,", "attend_row(q + ((b * Hq + h) * T) * d,"),
+    ("ring_slot", "long dst = ((b * Hkv + g) * W + pos % W) * d;",
+     "long dst = ((b * Hkv + g) * W + (pos + 1) % W) * d;"),
+    ("ring_window_short", "long lo = n > W ? n - W : 0;", "long lo = n > W ? n - W + 1 : 0;"),
+    ("ring_overwrite_order", "if (t_new - i > W) continue;", "if (i >= W) continue;"),
 ]
 
 
