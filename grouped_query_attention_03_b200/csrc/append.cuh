@@ -13,6 +13,11 @@
 //      2 x new bytes read + written).
 //   2. append_commit_kernel (one CTA): repeats the same check on the still
 //      unchanged lengths and, only if all are valid, advances them.
+//
+// ring != 0: a rolling buffer of C slots ("Relate shared heads to local
+// context": a rolling buffer that overwrites old KV entries), position p in
+// slot p mod C; of t_new new rows only the last C survive, and a length
+// only has to stay non-negative and inside int32.
 #pragma once
 
 #include "common.cuh"
@@ -20,12 +25,13 @@
 namespace gqa {
 
 __device__ __forceinline__ bool lengths_fit(const int32_t *seq_lens, int B,
-                                            int C, int t_new) {
-  // Block-wide: true iff every 0 <= len_b and len_b + t_new <= C.
+                                            int C, int t_new, int ring) {
+  // Block-wide: true iff every 0 <= len_b and len_b + t_new <= C (ring:
+  // len_b + t_new fits in int32).
   int bad = 0;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int n = seq_lens[b];
-    bad |= (n < 0 || n > C - t_new);
+    bad |= (n < 0 || n > (ring ? 0x7fffffff - t_new : C - t_new));
   }
   return __syncthreads_or(bad) == 0;
 }
@@ -37,8 +43,8 @@ __global__ void __launch_bounds__(256)
     append_copy_kernel(V *__restrict__ kc, V *__restrict__ vc,
                        const V *__restrict__ kn, const V *__restrict__ vn,
                        const int32_t *__restrict__ seq_lens, int B, int Hkv,
-                       int C, int t_new, int vec_per_row, int32_t *status) {
-  if (!lengths_fit(seq_lens, B, C, t_new)) {
+                       int C, int t_new, int vec_per_row, int ring, int32_t *status) {
+  if (!lengths_fit(seq_lens, B, C, t_new, ring)) {
     if (blockIdx.x == 0 && threadIdx.x == 0)
       record_status(status, GQA_ERR_CAPACITY);
     return;
@@ -52,15 +58,17 @@ __global__ void __launch_bounds__(256)
     const int i = (int)(row % t_new);
     const size_t lane = row / t_new;  // b * Hkv + g
     const int b = (int)(lane / Hkv);
-    const size_t dst = (lane * C + (size_t)(seq_lens[b] + i)) * vec_per_row + e;
+    if (ring && t_new - i > C) continue;  // overwritten by a later new row
+    const int cell = ring ? (int)(((long long)seq_lens[b] + i) % C) : seq_lens[b] + i;
+    const size_t dst = (lane * C + (size_t)cell) * vec_per_row + e;
     kc[dst] = kn[idx];
     vc[dst] = vn[idx];
   }
 }
 
 __global__ void __launch_bounds__(256)
-    append_commit_kernel(int32_t *seq_lens, int B, int C, int t_new) {
-  if (!lengths_fit(seq_lens, B, C, t_new)) return;
+    append_commit_kernel(int32_t *seq_lens, int B, int C, int t_new, int ring) {
+  if (!lengths_fit(seq_lens, B, C, t_new, ring)) return;
   for (int b = threadIdx.x; b < B; b += blockDim.x) seq_lens[b] += t_new;
 }
 

@@ -130,6 +130,8 @@ struct Params {
   int32_t *lens_out;
   int add;
   int lens_smem;  // 1: B <= kLensSmem, lengths cached in shared memory
+  int ring;       // 1: the cache is a rolling buffer of C slots, position p
+                  // in slot p mod C; the query reads all min(n_b, C) slots
 };
 
 // Keys of sequence b for this call (n_b, the appended token included).
@@ -145,9 +147,15 @@ __device__ __forceinline__ long long udiv(long long a, long long b) {
   return a / b;
 }
 
-__device__ __forceinline__ int eligible(int n, int window) {
-  return window > 0 ? min(n, window) : n;
+// Cells the query of a sequence with n positions reads: the window's last
+// cells, or (ring) every occupied slot [0, min(n, C)).
+__device__ __forceinline__ int eligible_cells(const Params &p, int n) {
+  return p.ring ? min(n, p.C) : (p.window > 0 ? min(n, p.window) : n);
 }
+__device__ __forceinline__ int first_cell(const Params &p, int n, int len) {
+  return p.ring ? 0 : n - len;
+}
+
 
 // Byte offset of 16-byte chunk `ch` (0..7) of row `r` inside a 128-byte
 // swizzled box (the TMA swizzle XORs the chunk index with r mod 8).
@@ -190,8 +198,8 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
   for (int b = lane; b < p.B; b += 32) {
     const int n = nlen(p, b);
     if (p.lens_smem) s_len[b] = n;
-    bad_local |= (n < p.add || n > p.C);
-    tot += eligible(max(n, 0), p.window);
+    bad_local |= (n < p.add || (!p.ring && n > p.C));
+    tot += eligible_cells(p, max(n, 0));
   }
   const bool bad = __any_sync(0xffffffffu, bad_local) != 0;
   if (lane == 0) *s_bad = bad ? 1 : 0;
@@ -214,7 +222,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     for (int b0 = 0; b0 < p.B && b < 0; b0 += 32) {
       const int bb = b0 + lane;
       const long long x =
-          bb < p.B ? (long long)eligible(len_of(bb), p.window) * p.VL : 0;
+          bb < p.B ? (long long)eligible_cells(p, len_of(bb)) * p.VL : 0;
       long long incl = x;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -231,8 +239,8 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
       }
     }
     int n_b = len_of(b);
-    int len = eligible(n_b, p.window);
-    int lo = n_b - len;
+    int len = eligible_cells(p, n_b);
+    int lo = first_cell(p, n_b, len);
     long long off0 = start - cum_b;
     int vl = (int)udiv(off0, len);
     int row = (int)(off0 - (long long)vl * len);
@@ -255,7 +263,9 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         h.slot = L + c;
         h.c0 = (int)udiv(SL, per);
         h.np = (int)udiv(SL + len - 1, per) - h.c0 + 1;
-        h.newrow = (p.add && row + nrows == len) ? nrows - 1 : -1;
+        // the appended token's cell: the last one, or (ring) its slot
+        const int cnew = p.ring ? (n_b - 1) % p.C : n_b - 1;
+        h.newrow = (p.add && cnew >= lo + row && cnew < lo + row + nrows) ? cnew - lo - row : -1;
         const int g = vl / p.nsub, sub = vl % p.nsub;
         const int h0 = g * p.r + sub * R;
         const int rc = min(R, p.r - sub * R);
@@ -300,15 +310,15 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
           int nb = -1;
           for (int b0 = b + 1; b0 < p.B && nb < 0 && pos < end; b0 += 32) {
             const int bb = b0 + lane;
-            const bool ne = bb < p.B && eligible(len_of(bb), p.window) > 0;
+            const bool ne = bb < p.B && eligible_cells(p, len_of(bb)) > 0;
             const unsigned m = __ballot_sync(0xffffffffu, ne);
             if (m) nb = b0 + __ffs(m) - 1;
           }
           if (nb < 0) break;
           b = nb;
           n_b = len_of(b);
-          len = eligible(n_b, p.window);
-          lo = n_b - len;
+          len = eligible_cells(p, n_b);
+          lo = first_cell(p, n_b, len);
         }
       }
     }

@@ -224,13 +224,13 @@ gqa_status launch_simt_decode(const void *q, const void *kc, const void *vc,
                               int Hkv, int C, int d, int window,
                               float scale_log2, int32_t *status,
                               cudaStream_t st, const void *kn = nullptr,
-                              const void *vn = nullptr, int add = 0) {
+                              const void *vn = nullptr, int add = 0, int ring = 0) {
   const dim3 grid(Hq, B);
   const int nf = (d + 31) / 32;
 #define GQA_DC(NF)                                                         \
   gqa::decode_simt_kernel<T, NF><<<grid, 32, 0, st>>>(                     \
       (const T *)q, (const T *)kc, (const T *)vc, (T *)o, lens, B, Hq, Hkv, \
-      C, d, window, scale_log2, status, (const T *)kn, (const T *)vn, add)
+      C, d, window, scale_log2, status, (const T *)kn, (const T *)vn, add, ring)
   switch (nf) {
     case 1: GQA_DC(1); break;
     case 2: GQA_DC(2); break;
@@ -391,11 +391,17 @@ size_t gqa_decode_workspace_bytes(gqa_dtype dtype, int B, int Hq, int Hkv,
 
 namespace {
 
+gqa_status append_impl(gqa_dtype dtype, void *k_cache, void *v_cache,
+                       const void *k_new, const void *v_new, int32_t *seq_lens,
+                       int B, int Hkv, int C, int d, int t_new, int ring,
+                       int32_t *dev_status, gqa_stream_t stream);
+
 // The fused append's extra operands (null for a plain decode).
 struct AppendArgs {
   void *k_cache, *v_cache;
   const void *k_new, *v_new;
   int32_t *seq_lens;
+  int ring;  // the cache is a rolling buffer of C slots
 };
 
 gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
@@ -462,6 +468,7 @@ gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
     p.lens_out = ap ? ap->seq_lens : nullptr;
     p.add = ap ? 1 : 0;
     p.lens_smem = B <= gqa::dec::kLensSmem ? 1 : 0;
+    p.ring = (ap && ap->ring) ? 1 : 0;
     if (cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;
@@ -475,18 +482,17 @@ gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
   // the append (same all-or-nothing length rule) writes them and advances
   // the lengths.
   const void *kn = ap ? ap->k_new : nullptr, *vn = ap ? ap->v_new : nullptr;
-  const int add = ap ? 1 : 0;
+  const int add = ap ? 1 : 0, ring = (ap && ap->ring) ? 1 : 0;
   s = dtype == GQA_F32
           ? launch_simt_decode<float>(q, k_cache, v_cache, o, seq_lens, B, Hq,
                                       Hkv, C, d, window, scale_log2,
-                                      dev_status, st, kn, vn, add)
+                                      dev_status, st, kn, vn, add, ring)
           : launch_simt_decode<bf16>(q, k_cache, v_cache, o, seq_lens, B, Hq,
                                      Hkv, C, d, window, scale_log2, dev_status,
-                                     st, kn, vn, add);
+                                     st, kn, vn, add, ring);
   if (s != GQA_OK || !ap) return s;
-  return gqa_cache_append(dtype, ap->k_cache, ap->v_cache, ap->k_new,
-                          ap->v_new, ap->seq_lens, B, Hkv, C, d, 1, dev_status,
-                          stream);
+  return append_impl(dtype, ap->k_cache, ap->v_cache, ap->k_new, ap->v_new,
+                     ap->seq_lens, B, Hkv, C, d, 1, ring, dev_status, stream);
 }
 
 }  // namespace
@@ -510,20 +516,38 @@ gqa_status gqa_decode_append(gqa_dtype dtype, const void *q, void *k_cache,
                              float scale, void *workspace,
                              size_t workspace_bytes, int32_t *dev_status,
                              gqa_stream_t stream) {
-  const AppendArgs ap{k_cache, v_cache, k_new, v_new, seq_lens};
+  const AppendArgs ap{k_cache, v_cache, k_new, v_new, seq_lens, 0};
   return decode_impl(dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, C, d,
                      window, scale, workspace, workspace_bytes, dev_status,
                      stream, &ap);
 }
 
-gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,
-                            const void *k_new, const void *v_new,
-                            int32_t *seq_lens, int B, int Hkv, int C, int d,
-                            int t_new, int32_t *dev_status,
-                            gqa_stream_t stream) {
+gqa_status gqa_ring_decode_append(gqa_dtype dtype, const void *q, void *k_ring,
+                                  void *v_ring, const void *k_new,
+                                  const void *v_new, void *o, int32_t *seq_lens,
+                                  int B, int Hq, int Hkv, int W, int d, float scale,
+                                  void *workspace, size_t workspace_bytes,
+                                  int32_t *dev_status, gqa_stream_t stream) {
+  if (W == 0) return GQA_ERR_SHAPE;
+  const AppendArgs ap{k_ring, v_ring, k_new, v_new, seq_lens, 1};
+  return decode_impl(dtype, q, k_ring, v_ring, o, seq_lens, B, Hq, Hkv, W, d,
+                     GQA_NO_WINDOW, scale, workspace, workspace_bytes, dev_status,
+                     stream, &ap);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Append t_new rows per sequence into a fixed-capacity cache (ring = 0) or
+// a rolling buffer of C slots (ring = 1, position p in slot p mod C).
+gqa_status append_impl(gqa_dtype dtype, void *k_cache, void *v_cache,
+                       const void *k_new, const void *v_new, int32_t *seq_lens,
+                       int B, int Hkv, int C, int d, int t_new, int ring,
+                       int32_t *dev_status, gqa_stream_t stream) {
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
   if (B < 0 || C < 0 || t_new < 0) return GQA_ERR_SHAPE;
-  if (Hkv <= 0 || d <= 0) return GQA_ERR_SHAPE;
+  if (Hkv <= 0 || d <= 0 || (ring && C == 0)) return GQA_ERR_SHAPE;
   const int esz = dtype == GQA_F32 ? 4 : 2;
   int64_t nc, nn;
   if (!elems(&nc, {B, Hkv, C, d, esz}) || !elems(&nn, {B, Hkv, t_new, d, esz}))
@@ -531,7 +555,7 @@ gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,
   if (B == 0 || t_new == 0) return GQA_OK;
   if (!k_cache || !v_cache || !k_new || !v_new || !seq_lens || !dev_status)
     return GQA_ERR_NULL;
-  if (t_new > C) return GQA_ERR_CAPACITY;
+  if (!ring && t_new > C) return GQA_ERR_CAPACITY;
   DeviceInfo di;
   gqa_status s = device_info(&di);
   if (s != GQA_OK) return s;
@@ -546,18 +570,39 @@ gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,
   if (vec)
     gqa::append_copy_kernel<uint4><<<grid, 256, 0, st>>>(
         (uint4 *)k_cache, (uint4 *)v_cache, (const uint4 *)k_new,
-        (const uint4 *)v_new, seq_lens, B, Hkv, C, t_new, vpr, dev_status);
+        (const uint4 *)v_new, seq_lens, B, Hkv, C, t_new, vpr, ring, dev_status);
   else if (esz == 4)
     gqa::append_copy_kernel<uint32_t><<<grid, 256, 0, st>>>(
         (uint32_t *)k_cache, (uint32_t *)v_cache, (const uint32_t *)k_new,
-        (const uint32_t *)v_new, seq_lens, B, Hkv, C, t_new, vpr, dev_status);
+        (const uint32_t *)v_new, seq_lens, B, Hkv, C, t_new, vpr, ring, dev_status);
   else
     gqa::append_copy_kernel<uint16_t><<<grid, 256, 0, st>>>(
         (uint16_t *)k_cache, (uint16_t *)v_cache, (const uint16_t *)k_new,
-        (const uint16_t *)v_new, seq_lens, B, Hkv, C, t_new, vpr, dev_status);
+        (const uint16_t *)v_new, seq_lens, B, Hkv, C, t_new, vpr, ring, dev_status);
   if (launch_status() != GQA_OK) return GQA_ERR_CUDA;
-  gqa::append_commit_kernel<<<1, 256, 0, st>>>(seq_lens, B, C, t_new);
+  gqa::append_commit_kernel<<<1, 256, 0, st>>>(seq_lens, B, C, t_new, ring);
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+gqa_status gqa_cache_append(gqa_dtype dtype, void *k_cache, void *v_cache,
+                            const void *k_new, const void *v_new,
+                            int32_t *seq_lens, int B, int Hkv, int C, int d,
+                            int t_new, int32_t *dev_status,
+                            gqa_stream_t stream) {
+  return append_impl(dtype, k_cache, v_cache, k_new, v_new, seq_lens, B, Hkv, C, d,
+                     t_new, 0, dev_status, stream);
+}
+
+gqa_status gqa_ring_append(gqa_dtype dtype, void *k_ring, void *v_ring,
+                           const void *k_new, const void *v_new, int32_t *seq_lens,
+                           int B, int Hkv, int W, int d, int t_new,
+                           int32_t *dev_status, gqa_stream_t stream) {
+  return append_impl(dtype, k_ring, v_ring, k_new, v_new, seq_lens, B, Hkv, W, d,
+                     t_new, 1, dev_status, stream);
 }
 
 }  // extern "C"

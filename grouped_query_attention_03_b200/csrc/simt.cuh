@@ -18,7 +18,8 @@ __device__ void attend_row_warp(const T *__restrict__ qrow,
                                 const T *__restrict__ klane,
                                 const T *__restrict__ vlane, int lo, int hi,
                                 int d, float scale_log2, T *__restrict__ orow,
-                                const T *kcand = nullptr, const T *vcand = nullptr) {
+                                const T *kcand = nullptr, const T *vcand = nullptr,
+                                int jcand = -1) {
   const int lane = threadIdx.x & 31;
   float q[NF], acc[NF];
 #pragma unroll
@@ -33,8 +34,9 @@ __device__ void attend_row_warp(const T *__restrict__ qrow,
     float s = -INFINITY;
     const int nk = min(32, hi - j0 + 1);
     for (int jj = 0; jj < nk; ++jj) {
-      // Key `hi` may be a candidate row held outside the lane (fused append).
-      const T *kr = (kcand && j0 + jj == hi) ? kcand : klane + (size_t)(j0 + jj) * d;
+      // Key `jcand` may be a candidate row held outside the lane (fused
+      // append).
+      const T *kr = (kcand && j0 + jj == jcand) ? kcand : klane + (size_t)(j0 + jj) * d;
       float part = 0.f;
 #pragma unroll
       for (int i = 0; i < NF; ++i) {
@@ -63,7 +65,7 @@ __device__ void attend_row_warp(const T *__restrict__ qrow,
     for (int i = 0; i < NF; ++i) acc[i] *= alpha;
     for (int jj = 0; jj < nk; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const T *vr = (vcand && j0 + jj == hi) ? vcand : vlane + (size_t)(j0 + jj) * d;
+      const T *vr = (vcand && j0 + jj == jcand) ? vcand : vlane + (size_t)(j0 + jj) * d;
 #pragma unroll
       for (int i = 0; i < NF; ++i) {
         const int f = lane + 32 * i;
@@ -153,13 +155,13 @@ __global__ void __launch_bounds__(32)
                        const int32_t *__restrict__ seq_lens, int B, int Hq,
                        int Hkv, int C, int d, int window, float scale_log2,
                        int32_t *status, const T *kn = nullptr,
-                       const T *vn = nullptr, int add = 0) {
+                       const T *vn = nullptr, int add = 0, int ring = 0) {
   const int h = blockIdx.x, b = blockIdx.y;
   T *orow = o + ((size_t)b * Hq + h) * d;
   bool bad = false;
   for (int i = threadIdx.x; i < B; i += 32) {
     const int n = seq_lens[i] + add;
-    bad |= (n < add || n > C);
+    bad |= (n < add || (!ring && n > C));
   }
   if (__any_sync(0xffffffffu, bad)) {
     if (threadIdx.x == 0 && b == 0 && h == 0)
@@ -173,13 +175,16 @@ __global__ void __launch_bounds__(32)
     return;
   }
   const int r = Hq / Hkv, g = h / r;
-  const int pos = n - 1;
-  const int lo = window > 0 ? max(0, pos - (window - 1)) : 0;
+  // Linear: cells [max(0, n-w), n), the newest last.  Ring (rolling buffer
+  // of C slots): every occupied slot, the newest at slot (n-1) mod C.
+  const int pos = ring ? min(n, C) - 1 : n - 1;
+  const int lo = (!ring && window > 0) ? max(0, pos - (window - 1)) : 0;
   const size_t lane_off = ((size_t)b * Hkv + g) * C * d;
   const size_t cand = ((size_t)b * Hkv + g) * d;
   attend_row_warp<T, NF>(q + ((size_t)b * Hq + h) * d, kc + lane_off,
                          vc + lane_off, lo, pos, d, scale_log2, orow,
-                         add ? kn + cand : nullptr, add ? vn + cand : nullptr);
+                         add ? kn + cand : nullptr, add ? vn + cand : nullptr,
+                         ring ? (n - 1) % C : pos);
 }
 
 }  // namespace gqa

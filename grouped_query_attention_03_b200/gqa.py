@@ -28,7 +28,7 @@ STATUS_NAMES = {
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_prefill", "gqa_prefill_packed", "gqa_decode", "gqa_decode_workspace_bytes",
            "gqa_decode_append", "gqa_decode_multi", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
-           "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
+           "gqa_ring_append", "gqa_ring_decode_append", "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
            "gqa_version")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # GQA_NOALLOC_SCRATCH_BYTES in include/gqa.h
@@ -75,6 +75,10 @@ def _declare(L):
     L.gqa_decode_workspace_bytes.restype = sz
     L.gqa_cache_append.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 5 + [vp, vp]
     L.gqa_cache_append.restype = i32
+    L.gqa_ring_append.argtypes = [i32, vp, vp, vp, vp, vp] + [i32] * 5 + [vp, vp]
+    L.gqa_ring_append.restype = i32
+    L.gqa_ring_decode_append.argtypes = [i32] + [vp] * 7 + [i32] * 5 + [f32, vp, sz, vp, vp]
+    L.gqa_ring_decode_append.restype = i32
     L.gqa_cache_bytes.argtypes = [i64] * 6
     L.gqa_cache_bytes.restype = ctypes.c_uint64
     L.gqa_kv_head_for_query.argtypes = [i32] * 3
@@ -131,6 +135,52 @@ def _stream(stream, device):
 
 def _window(window):
     return NO_WINDOW if window is None else int(window)
+
+
+def ring_append(k_ring, v_ring, k_new, v_new, seq_lens, *, status=None, stream=None):
+    """Rolling buffer of W slots (k_ring [B,Hkv,W,d]): write positions
+    [len_b, len_b + t_new) at slots p mod W (the last W of them survive) and
+    advance seq_lens in place."""
+    B, Hkv, W, d = k_ring.shape
+    t_new = k_new.shape[2]
+    if k_new.shape != (B, Hkv, t_new, d) or v_new.shape != k_new.shape:
+        raise ValueError("new K/V shape mismatch")
+    dev = k_ring.device
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_ring_append(
+        _dtype_code(k_ring), _ptr(k_ring, "k_ring"), _ptr(v_ring, "v_ring", k_ring.dtype, dev),
+        _ptr(k_new, "k_new", k_ring.dtype, dev), _ptr(v_new, "v_new", k_ring.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hkv, W, d, t_new,
+        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_ring_append")
+
+
+def ring_decode_append(q, k_ring, v_ring, k_new, v_new, seq_lens, *, scale=None, out=None,
+                       workspace=None, status=None, stream=None):
+    """The decode step against a rolling buffer of W slots, the step's row
+    appended in the same call: the query at position len_b reads the last W
+    positions; seq_lens (positions before the step) grows by one."""
+    B, Hq, d = q.shape
+    Hkv, W = k_ring.shape[1], k_ring.shape[2]
+    if k_ring.shape != (B, Hkv, W, d) or v_ring.shape != k_ring.shape:
+        raise ValueError("ring shape mismatch")
+    if k_new.shape != (B, Hkv, 1, d) or v_new.shape != k_new.shape:
+        raise ValueError("new K/V must be [B,Hkv,1,d]")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    dev = q.device
+    if workspace is None:
+        workspace = decode_workspace(q, k_ring)
+    st = new_status(dev) if status is None else status
+    _check(lib().gqa_ring_decode_append(
+        _dtype_code(q), _ptr(q, "q"), _ptr(k_ring, "k_ring", q.dtype, dev),
+        _ptr(v_ring, "v_ring", q.dtype, dev), _ptr(k_new, "k_new", q.dtype, dev),
+        _ptr(v_new, "v_new", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, W, d, float(scale),
+        _ptr(workspace, "workspace", torch.uint8, dev), workspace.numel(),
+        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_ring_decode_append")
+    return out
 
 
 def new_status(device):

@@ -214,6 +214,43 @@ gqa_status gqa_decode_multi(gqa_dtype dtype, const void *q, const void *k_cache,
                             int window, float scale, int32_t *dev_status,
                             gqa_stream_t stream);
 
+/*
+ * Rolling-buffer (ring) cache.  [P1] "Relate shared heads to local context"
+ * describes Mistral's rolling buffer that overwrites old KV entries (the
+ * chapter itself keeps every row and does not build one).  Here a ring of
+ * W slots per KV lane holds position p in slot p mod W, so it always holds
+ * the last W positions: attending over it is the window-W decode of
+ * [P1] "Intersect the window ..." with W cells of storage instead of the
+ * whole prefix.  seq_lens counts positions so far (not capped at W).
+ *
+ * gqa_ring_append -- write positions [len_b, len_b + t_new) (k_new, v_new
+ *   [B,Hkv,t_new,d]; only the last W rows survive) into k_ring/v_ring
+ *   [B,Hkv,W,d] and advance seq_lens.  A negative length, or one that would
+ *   pass INT32_MAX, sets *dev_status to GQA_ERR_CAPACITY and nothing moves.
+ */
+gqa_status gqa_ring_append(gqa_dtype dtype, void *k_ring, void *v_ring,
+                           const void *k_new, const void *v_new, int32_t *seq_lens,
+                           int B, int Hkv, int W, int d, int t_new,
+                           int32_t *dev_status, gqa_stream_t stream);
+
+/*
+ * gqa_ring_decode_append -- the decode step against a ring, with the step's
+ * row appended in the same call (as gqa_decode_append): seq_lens[b] =
+ * positions before the step; the query at position len_b reads positions
+ * [max(0, len_b + 1 - W), len_b] (every occupied slot, the new one read
+ * from k_new / v_new [B,Hkv,1,d] and written to slot len_b mod W); then
+ * len_b grows by one.  Workspace: gqa_decode_workspace_bytes(dtype, B, Hq,
+ * Hkv, W, d).  A negative length sets GQA_ERR_CAPACITY, zeroes the output
+ * and changes nothing.  bf16 with d in {64, 128} runs the split-K kernel;
+ * other d and fp32 run on CUDA cores.
+ */
+gqa_status gqa_ring_decode_append(gqa_dtype dtype, const void *q, void *k_ring,
+                                  void *v_ring, const void *k_new,
+                                  const void *v_new, void *o, int32_t *seq_lens,
+                                  int B, int Hq, int Hkv, int W, int d, float scale,
+                                  void *workspace, size_t workspace_bytes,
+                                  int32_t *dev_status, gqa_stream_t stream);
+
 /* Size of the fixed device array gqa_decode_noalloc uses as its workspace. */
 #define GQA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 

@@ -151,6 +151,39 @@ def test_prefill_packed_host_refusals(L):
     assert f(*empty) == OK
 
 
+def test_ring_host_refusals(L):
+    # gqa_ring_append(dtype, k, v, kn, vn, lens, B, Hkv, W, d, t_new, status, stream)
+    ra = [1, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 4, 64, 9, FAKE, None]
+    w0 = list(ra)
+    w0[8] = 0
+    assert L.gqa_ring_append(*w0) == SHAPE
+    neg = list(ra)
+    neg[10] = -1
+    assert L.gqa_ring_append(*neg) == SHAPE
+    nolens = list(ra)
+    nolens[5] = None
+    assert L.gqa_ring_append(*nolens) == NULL
+    empty = list(ra)
+    empty[10] = 0
+    assert L.gqa_ring_append(*empty) == OK
+    # gqa_ring_decode_append(dtype, q, kr, vr, kn, vn, o, lens, B, Hq, Hkv, W, d, scale,
+    #                        ws, wsb, status, stream)
+    rd = [1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 8, 64, 0.125, FAKE, 1 << 30,
+          FAKE, None]
+    w0 = list(rd)
+    w0[11] = 0
+    assert L.gqa_ring_decode_append(*w0) == SHAPE
+    groups = list(rd)
+    groups[9] = 3
+    assert L.gqa_ring_decode_append(*groups) == GROUPS
+    nokn = list(rd)
+    nokn[4] = None
+    assert L.gqa_ring_decode_append(*nokn) == NULL
+    nows = list(rd)
+    nows[14] = None
+    assert L.gqa_ring_decode_append(*nows) == 8
+
+
 def test_prefill_host_refusals(L):
     assert _prefill(L, Hq=6, Hkv=4) == GROUPS
     assert _prefill(L, Hkv=0) == SHAPE
