@@ -133,14 +133,14 @@ def dist_max(x, device):
 # changes the figure no longer describes the kernel and is reported as null.
 CAPTURED_TRAFFIC = {
     ("decode_b8_n8000", "decode"): {
-        "bytes": 269_470_464, "window": None, "hkv": None,
+        "bytes": 268_979_200, "window": None, "hkv": None,
         "sources": ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "6ee46a78e5b230c58fb9262b4194bbb95a94ab4a8faaae38a819350ffda2fcd7",
+        "sha256": "8aff895ca79dff537dd6e24f0ca19d319fd2cb0e18c05b59360b4f257824d918",
         "profile": "profiles/decode_split_kernel_b8_n8000.md"},
     ("swa_t32768", "prefill"): {
-        "bytes": 714_170_624, "window": 4096, "hkv": None,
+        "bytes": 698_675_200, "window": 4096, "hkv": None,
         "sources": ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "7dfc2df64633b728d62493bc0ac980655e3bea0a3b1fc0893e268a1f383813d0",
+        "sha256": "a1d191a5db57ed82de0191eee5a8e1769893e6c34dbc55d58ac50ba236e8d5ae",
         "profile": "profiles/prefill_pair_kernel_swa_t32768.md"},
 }
 
