@@ -15,15 +15,19 @@
 //               S_A(0), S_B(0), then per KV tile j:
 //               O_A += P_A(j) V_j, S_A(j+1), O_B += P_B(j) V_j, S_B(j+1)
 //               so the tensor pipe runs one head while the other head's
-//               softmax warps work.
+//               softmax warps work.  P V takes P from TMEM (A operand) and
+//               V from shared memory; S(j+1) overwrites P(j) only after
+//               P V(j), since one thread's MMAs execute in issue order.
 //   warps 2-3   idle (they complete the first warpgroup, which hands most of
 //               its registers to the softmax warpgroups with setmaxnreg).
 //   warps 4-7   softmax of head A, warps 8-11 softmax of head B: thread = row
 //               (TMEM lane); the whole 128-score row is read from TMEM into
 //               registers at once, then row max, lazy O rescale, and bf16 P
-//               written to shared memory (K-major, 128-byte swizzle); O / l
-//               epilogue.
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+d), O_B after it.
+//               written back to the same TMEM lane over the first 64 S
+//               columns (no shared-memory round trip for P); O / l epilogue.
+// TMEM columns: S_A [0,128) (P_A in [0,64)), S_B [128,256) (P_B in
+// [128,192)), O_A [256, 256+d), O_B after it.  Shared memory holds the two
+// Q tiles and the K/V ring only.
 #pragma once
 
 #include <cuda.h>
@@ -42,6 +46,7 @@ constexpr int kThreads = 384;
 // 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * (launch registers).
 constexpr int kRegsLow = 72, kRegsHigh = 216;
 constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxSlots = 12;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -49,14 +54,13 @@ struct Cfg {
   static constexpr int KB = D / 64;                  // 64-column blocks
   static constexpr int BLK = kBM * 128;              // 128 rows x 128 B
   static constexpr int TILE = KB * BLK;              // a Q, K or V tile
-  static constexpr int NSLOT = (D == 128) ? 3 : 6;   // K/V ring slots
+  static constexpr int NSLOT = (D == 128) ? 3 : 6;   // K/V ring slots (deeper measured no faster)
   static constexpr int OFF_QA = 0;
   static constexpr int OFF_QB = TILE;
   static constexpr int OFF_RING = 2 * TILE;
-  static constexpr int OFF_PA = OFF_RING + NSLOT * TILE;
-  static constexpr int P_BYTES = kBM * kBN * 2;
-  static constexpr int OFF_PB = OFF_PA + P_BYTES;
-  static constexpr int SMEM = OFF_PB + P_BYTES + 1024;
+  static constexpr int SMEM = OFF_RING + NSLOT * TILE + 1024;  // + alignment slack
+  static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  static_assert(NSLOT <= kMaxSlots, "ring barriers");
   static constexpr uint32_t TM_O = 256;              // O_A column; O_B = TM_O + D
 };
 
@@ -89,7 +93,7 @@ __device__ __forceinline__ int row_lo(const Params &p, int b, int t) {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t full[6], empty[6];
+  uint64_t full[kMaxSlots], empty[kMaxSlots];
   uint64_t s_full[2], p_full[2], o_done[2];
   uint64_t mma_fin;
   uint64_t v_clean;  // the last V tile's rows past the sequence are zero
@@ -112,30 +116,27 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 }
 
 // p = 2^(s*scale - m) for this thread's row of kBN scores (special-function
-// unit; masked cells give exactly 0), written as bf16 P (K-major, 128-byte
-// swizzle, 16-byte chunks); returns the row sum.
+// unit; masked cells give exactly 0), written as bf16 P into this thread's
+// TMEM lane over the S columns it came from (column c holds p[2c], p[2c+1]),
+// where the P V MMA reads it as its A operand; returns the row sum.
 template <int D>
-__device__ __forceinline__ float emit_p(const float *s, float sc, float m, unsigned char *sP,
-                                        int row) {
-  using K = Cfg<D>;
+__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP) {
   float2 lsum2 = make_float2(0.f, 0.f);
   const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
 #pragma unroll
-  for (int chunk = 0; chunk < kBN / 8; ++chunk) {
-    uint32_t w4[4];
+  for (int half = 0; half < 2; ++half) {
+    float w[32];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int i = chunk * 8 + 2 * e;
+    for (int e = 0; e < 32; ++e) {
+      const int i = half * 64 + 2 * e;
       const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
       const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       lsum2 = fadd2v(lsum2, pv);
-      w4[e] = pack_bf16(pv.x, pv.y);
+      w[e] = __uint_as_float(pack_bf16(pv.x, pv.y));
     }
-    const int blk = chunk >> 3, cc = chunk & 7;
-    unsigned char *dst = sP + blk * K::BLK + (row >> 3) * 1024 + (row & 7) * 128 +
-                         ((cc ^ (row & 7)) << 4);
-    *reinterpret_cast<uint4 *>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    tc::tmem_st32(tP + half * 32, w);
   }
+  tc::tmem_wait_st();
   return lsum2.x + lsum2.y;
 }
 
@@ -158,7 +159,6 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
   const uint32_t tS = tmem + lane_base + hd * kBN;
   const uint32_t tO = tmem + lane_base + K::TM_O + hd * D;
   const float sc = p.scale_log2;
-  unsigned char *sP = smem + (hd ? K::OFF_PB : K::OFF_PA);
   float m_run = -INFINITY, l_run = 0.f;
   bool ok = true;
   for (int j = 0; j < nt; ++j) {
@@ -211,9 +211,8 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
       l_run *= alpha;
       m_run = m_new;
     }
-    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, sP, row);
+    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS);
     l_run += lsum;
-    tc::fence_proxy_async_smem();
     tc::fence_before_sync();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars.p_full[hd]);
@@ -418,7 +417,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t sQ[2] = {smem_u32(smem + K::OFF_QA), smem_u32(smem + K::OFF_QB)};
-      const uint32_t sP[2] = {smem_u32(smem + K::OFF_PA), smem_u32(smem + K::OFF_PB)};
       auto slot_addr = [&](int i) { return smem_u32(smem + K::OFF_RING + (i % K::NSLOT) * K::TILE); };
       auto wait_load = [&](int i) {
         return mbar_wait(&bars.full[i % K::NSLOT], (i / K::NSLOT) & 1, &failed);
@@ -434,12 +432,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_commit(&bars.s_full[hd]);
       };
       auto issue_pv = [&](int hd, int j) {
+        // A = P from TMEM (over S of this head: 8 columns per 16 keys)
         const uint32_t sV = slot_addr(2 * j + 1);
 #pragma unroll
         for (int k = 0; k < kBN / 16; ++k) {
-          const uint64_t da = tc::sw128_desc(sP[hd] + (k >> 2) * K::BLK + (k & 3) * 32, 16, 1024);
           const uint64_t db = tc::sw128_desc(sV + k * 16 * 128, K::BLK, 1024);
-          tc::mma_bf16_ss(tmem + K::TM_O + hd * D, da, db, idO, (j > 0 || k > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tmem + K::TM_O + hd * D, tmem + hd * kBN + k * 8, db, idO,
+                          (j > 0 || k > 0) ? 1u : 0u);
         }
         tc::mma_commit(&bars.o_done[hd]);
       };
