@@ -174,6 +174,13 @@ __device__ __forceinline__ void ffma2(float2 &d, float2 a, float2 b) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x with the special-function unit's instruction (ex2.approx.ftz.f32:
 // results below the normal range flush to zero, so 2^-inf = 0).
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -193,7 +193,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
       float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (!neg) {
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) mc[i & 3] = fmaxf(mc[i & 3], s[i]);
+        for (int i = 0; i < kBN; i += 2) mc[(i >> 1) & 3] = fmax3(mc[(i >> 1) & 3], s[i], s[i + 1]);
       } else {
 #pragma unroll
         for (int i = 0; i < kBN; ++i)
