@@ -661,10 +661,14 @@ __device__ void consumer(const Params &p, unsigned char *smem,
               out[h * D + lane + 32 * k] = __float2bfloat16_rn(a[k] * inv);
           }
         } else {
+          // The lane's merge reads this partial at the end of the kernel,
+          // after the rest of the cache has streamed through L2: keep it.
+          const uint64_t keep = tc::l2_policy_evict_last();
 #pragma unroll
           for (int k = 0; k < D / 32; ++k)
-            p.acc[((size_t)hd.slot * R + h) * D + lane + 32 * k] = a[k];
-          if (lane == 0) p.ml[(size_t)hd.slot * R + h] = make_float2(mm, lsum);
+            tc::st_global_hint(&p.acc[((size_t)hd.slot * R + h) * D + lane + 32 * k], a[k], keep);
+          if (lane == 0)
+            tc::st_global_hint(&p.ml[(size_t)hd.slot * R + h], make_float2(mm, lsum), keep);
         }
       }
       // A partial is counted at the end of the CTA's range: nobody needs it

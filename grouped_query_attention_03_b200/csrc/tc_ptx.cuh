@@ -206,6 +206,25 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   return pol;
 }
 
+// An L2 cache policy that evicts last: for small data read again later in
+// the same kernel after a large stream has passed through L2.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 32-bit global store with an L2 cache policy.
+__device__ __forceinline__ void st_global_hint(float *addr, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(addr), "f"(v), "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ void st_global_hint(float2 *addr, float2 v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(addr), "f"(v.x),
+               "f"(v.y), "l"(policy)
+               : "memory");
+}
+
 // tma_load_2d with an L2 cache policy.
 __device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorMap *map,
                                                  int c0, int c1, uint64_t *bar,
