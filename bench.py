@@ -133,14 +133,14 @@ def dist_max(x, device):
 # changes the figure no longer describes the kernel and is reported as null.
 CAPTURED_TRAFFIC = {
     ("decode_b8_n8000", "decode"): {
-        "bytes": 268_979_200, "window": None, "hkv": None,
+        "bytes": 268_659_712, "window": None, "hkv": None,
         "sources": ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "8aff895ca79dff537dd6e24f0ca19d319fd2cb0e18c05b59360b4f257824d918",
+        "sha256": "28b96ea410947a12049e6cb02cb90f4eba0af835b8ea9b7abaaa79562a6d5aab",
         "profile": "profiles/decode_split_kernel_b8_n8000.md"},
     ("swa_t32768", "prefill"): {
-        "bytes": 698_675_200, "window": 4096, "hkv": None,
+        "bytes": 692_894_976, "window": 4096, "hkv": None,
         "sources": ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "a1d191a5db57ed82de0191eee5a8e1769893e6c34dbc55d58ac50ba236e8d5ae",
+        "sha256": "1c048c911b18fbbb614c0d38605bc0f0c4d62456b0cebb82bffc519eb39dd8cd",
         "profile": "profiles/prefill_pair_kernel_swa_t32768.md"},
 }
 
