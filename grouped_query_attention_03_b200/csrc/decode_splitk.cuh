@@ -132,6 +132,7 @@ struct Params {
   int lens_smem;  // 1: B <= kLensSmem, lengths cached in shared memory
   int ring;       // 1: the cache is a rolling buffer of C slots, position p
                   // in slot p mod C; the query reads all min(n_b, C) slots
+  int pad;        // virtual rows in front of every non-empty lane (below)
 };
 
 // Keys of sequence b for this call (n_b, the appended token included).
@@ -154,6 +155,13 @@ __device__ __forceinline__ int eligible_cells(const Params &p, int n) {
 }
 __device__ __forceinline__ int first_cell(const Params &p, int n, int len) {
   return p.ring ? 0 : n - len;
+}
+// A lane's share of the row space the CTAs split: its rows plus `pad`
+// virtual rows in front of them that carry no work.  A lane segment costs a
+// CTA a fixed amount of work (query load, combine, partial), so a range
+// that starts a lane gets that many fewer real rows.
+__device__ __forceinline__ int extent(const Params &p, int len) {
+  return len > 0 ? len + p.pad : 0;
 }
 
 
@@ -199,7 +207,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     const int n = nlen(p, b);
     if (p.lens_smem) s_len[b] = n;
     bad_local |= (n < p.add || (!p.ring && n > p.C));
-    tot += eligible_cells(p, max(n, 0));
+    tot += extent(p, eligible_cells(p, max(n, 0)));
   }
   const bool bad = __any_sync(0xffffffffu, bad_local) != 0;
   if (lane == 0) *s_bad = bad ? 1 : 0;
@@ -222,7 +230,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     for (int b0 = 0; b0 < p.B && b < 0; b0 += 32) {
       const int bb = b0 + lane;
       const long long x =
-          bb < p.B ? (long long)eligible_cells(p, len_of(bb)) * p.VL : 0;
+          bb < p.B ? (long long)extent(p, eligible_cells(p, len_of(bb))) * p.VL : 0;
       long long incl = x;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -240,16 +248,22 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
     }
     int n_b = len_of(b);
     int len = eligible_cells(p, n_b);
+    int ext = extent(p, len);
     int lo = first_cell(p, n_b, len);
     long long off0 = start - cum_b;
-    int vl = (int)udiv(off0, len);
-    int row = (int)(off0 - (long long)vl * len);
+    int vl = (int)udiv(off0, ext);
+    int row = (int)(off0 - (long long)vl * ext) - p.pad;  // < 0: in the padding
     long long pos = start;
     bool seg_first = true;
 
     while (pos < end) {
+      if (row < 0) {  // skip the lane's virtual rows
+        pos -= row;
+        row = 0;
+        if (pos >= end) break;
+      }
       const int L = b * p.VL + vl;
-      const long long SL = cum_b + (long long)vl * len;
+      const long long SR = cum_b + (long long)vl * ext + p.pad;  // first real row
       const int nrows = (int)min((long long)min(K::ROWS, len - row), end - pos);
       const bool last = (row + nrows == len) || (pos + nrows == end);
       int st;
@@ -261,8 +275,8 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         h.nrows = nrows;
         h.flags = (seg_first ? kFirst : 0) | (last ? kLast : 0);
         h.slot = L + c;
-        h.c0 = (int)udiv(SL, per);
-        h.np = (int)udiv(SL + len - 1, per) - h.c0 + 1;
+        h.c0 = (int)udiv(SR, per);
+        h.np = (int)udiv(SR + len - 1, per) - h.c0 + 1;
         // the appended token's cell: the last one, or (ring) its slot
         const int cnew = p.ring ? (n_b - 1) % p.C : n_b - 1;
         h.newrow = (p.add && cnew >= lo + row && cnew < lo + row + nrows) ? cnew - lo - row : -1;
@@ -302,10 +316,10 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
       row += nrows;
       seg_first = last;
       if (row == len) {
-        row = 0;
+        row = -p.pad;
         if (++vl == p.VL) {
           vl = 0;
-          cum_b += (long long)len * p.VL;
+          cum_b += (long long)ext * p.VL;
           // Next batch row with a non-empty range (warp-parallel search).
           int nb = -1;
           for (int b0 = b + 1; b0 < p.B && nb < 0 && pos < end; b0 += 32) {
@@ -318,6 +332,7 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
           b = nb;
           n_b = len_of(b);
           len = eligible_cells(p, n_b);
+          ext = extent(p, len);
           lo = first_cell(p, n_b, len);
         }
       }

@@ -29,6 +29,12 @@ constexpr int kMaxDecodeCtas = 1024;  // workspace is sized for this many
 #define GQA_DEC_MIN_ROWS 256
 #endif
 constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;  // smallest row range per CTA
+#ifndef GQA_DEC_LANE_PAD_BYTES
+#define GQA_DEC_LANE_PAD_BYTES 65536
+#endif
+// A lane segment's fixed cost in a CTA, as cache bytes: the split gives each
+// non-empty lane this many bytes of virtual rows (see dec::extent).
+constexpr int kDecodeLanePadBytes = GQA_DEC_LANE_PAD_BYTES;
 
 struct DeviceInfo {
   int sms = 0;
@@ -469,6 +475,7 @@ gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
     p.add = ap ? 1 : 0;
     p.lens_smem = B <= gqa::dec::kLensSmem ? 1 : 0;
     p.ring = (ap && ap->ring) ? 1 : 0;
+    p.pad = kDecodeLanePadBytes / (4 * d);  // K and V rows of d bf16
     if (cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;
