@@ -30,7 +30,7 @@ constexpr int kMaxDecodeCtas = 1024;  // workspace is sized for this many
 #endif
 constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;  // smallest row range per CTA
 #ifndef GQA_DEC_LANE_PAD_BYTES
-#define GQA_DEC_LANE_PAD_BYTES 65536
+#define GQA_DEC_LANE_PAD_BYTES 131072
 #endif
 // A lane segment's fixed cost in a CTA, as cache bytes: the split gives each
 // non-empty lane this many bytes of virtual rows (see dec::extent).

@@ -91,7 +91,7 @@ def test_split_plan_random_length_mixes():
 
 
 def test_split_plan_workload_shapes():
-    check([8001] * 8, 8, 148, 256, 128)                       # the B=8 decode
+    check([8001] * 8, 8, 148, 256, 256)                       # the B=8 decode
     rng = random.Random(3)
     check([rng.randint(2, 8193) for _ in range(64)], 1, 148, 256, 128)   # ragged MQA
     check([4096], 8, 148, 256, 128)                           # window-4096 step
