@@ -279,11 +279,12 @@ class DecodeStep:
 class PrefillStep:
     """One gqa_prefill over a whole prompt batch."""
 
-    def __init__(self, w, device, window):
+    def __init__(self, w, device, window, Hkv=None):
         from grouped_query_attention_03_b200 import gqa
         self.gqa, self.w, self.window = gqa, w, window
+        self.Hkv = Hkv or w.Hkv
         self.q, self.k, self.v = [t.to(device) for t in synthetic.qkv_prefill(
-            w.B, w.Hq, w.Hkv, w.T, w.d, w.seed, std=w.std)]
+            w.B, w.Hq, self.Hkv, w.T, w.d, w.seed, std=w.std)]
         self.o = torch.empty_like(self.q)
         t = np.arange(w.T)
         lo = np.maximum(0, t - (window - 1)) if window else np.zeros_like(t)
@@ -296,21 +297,21 @@ class PrefillStep:
 
     def describe(self):
         w = self.w
-        return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T,
+        return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": self.Hkv, "d": w.d, "T": w.T,
                 "window": self.window, "permitted_pairs_per_head": self.pairs}
 
     def kernel(self):
         """The tensor-core kernel gqa_prefill dispatches to for this shape."""
         w = self.w
-        if w.d in (64, 128) and (w.Hq // w.Hkv) % 2 == 0:
+        if w.d in (64, 128) and (w.Hq // self.Hkv) % 2 == 0:
             return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
         return "pf::prefill_kernel (one query head per CTA)"
 
 
-def measure_prefill(w, window, device, reps, warmup):
+def measure_prefill(w, window, device, reps, warmup, Hkv=None):
     """Per-launch prefill time (CUDA events), L2 flushed between launches
     when the inputs fit in L2."""
-    step = PrefillStep(w, device, window)
+    step = PrefillStep(w, device, window, Hkv)
     flush = make_flush(device) if step.in_bytes <= 126e6 else None
     for _ in range(warmup):
         step.run()
@@ -562,7 +563,7 @@ def run_gpu_prefill(args, world, rank, local):
     window = args.window if args.window is not None else w.windows[0]
     barrier()
     with ClockSampler(local) as clocks:
-        step, res = measure_prefill(w, window, device, args.steps, args.warmup)
+        step, res = measure_prefill(w, window, device, args.steps, args.warmup, args.hkv)
     ms = dist_max(res["ms"], device)
     peaks, kind = measured_peaks()
     value = aggregate_rate(step.flops, 1, world, ms) / 1e12

@@ -21,9 +21,9 @@
 //   warps 2-5   softmax: thread = query row (TMEM lane); tcgen05.ld of the S
 //               row, causal/window mask on edge tiles only, online max with
 //               lazy O rescaling (only when the max grows by more than 2^8),
-//               P in bf16 to shared memory (128-byte swizzled K-major layout
-//               for the PV MMA), then the O / l epilogue.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d).
+//               P in bf16 to TMEM (the PV MMA takes its A operand from
+//               there), then the O / l epilogue.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d), P [256+d, 320+d).
 #pragma once
 
 #include <cuda.h>
@@ -49,9 +49,11 @@ struct Cfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
-  static constexpr int OFF_P = OFF_V + STAGES * TILE;
-  static constexpr int P_BYTES = kBM * kBN * 2;
-  static constexpr int DYN_BYTES = OFF_P + P_BYTES;
+  static constexpr int DYN_BYTES = OFF_V + STAGES * TILE;
+  // TMEM columns: S double buffer [0, 256), O [256, 256 + D), and P (bf16,
+  // two keys per 32-bit column) in the 64 columns after O.
+  static constexpr uint32_t TM_P = 256 + D;
+  static_assert(TM_P + kBN / 2 <= kTmemCols, "S, O and P must fit in 512 TMEM columns");
   // Ask for at least 120 KB so only one CTA (which holds all 512 TMEM
   // columns) is resident per SM.
   static constexpr int SMEM = (DYN_BYTES + 1024 > 120 * 1024 ? DYN_BYTES + 1024 : 120 * 1024);
@@ -233,17 +235,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
       const uint32_t sQ = smem_u32(smem + K::OFF_Q);
-      const uint32_t sP = smem_u32(smem + K::OFF_P);
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait(&bars.p_full, i & 1, &failed)) return false;
         if (!mbar_wait(&bars.v_full[i & 1], (i >> 1) & 1, &failed)) return false;
         tc::fence_after_sync();
         const uint32_t sV = smem_u32(smem + K::OFF_V + (i & 1) * K::TILE);
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
-          const uint64_t da = tc::sw128_desc(sP + (k >> 2) * K::BLK + (k & 3) * 32, 16, 1024);
+        for (int k = 0; k < kBN / 16; ++k) {  // A = P from TMEM, 8 columns per 16 keys
           const uint64_t db = tc::sw128_desc(sV + k * 16 * 128, K::BLK, 1024);
-          tc::mma_bf16_ss(tmem + 256, da, db, idO, (i > 0 || k > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tmem + 256, tmem + K::TM_P + k * 8, db, idO, (i > 0 || k > 0) ? 1u : 0u);
         }
         tc::mma_commit(&bars.o_done);
         tc::mma_commit(&bars.v_empty[i & 1]);
@@ -286,7 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lo_t = active ? row_lo(p, b, t) : 0;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const float sc = p.scale_log2;
-    unsigned char *sP = smem + K::OFF_P;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -355,23 +354,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_run = m_new;
       }
       const float msub = m_run == -INFINITY ? 0.f : m_run;
+      // bf16 P into this thread's TMEM lane (column c holds p[2c], p[2c+1]),
+      // where the P V MMA reads it as its A operand.
       float lsum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kBN / 8; ++c) {
-        uint32_t w4[4];
+      for (int half = 0; half < 2; ++half) {
+        float w[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2_approx(fmaf(s[c * 8 + 2 * e], sc, -msub));
-          const float p1 = ex2_approx(fmaf(s[c * 8 + 2 * e + 1], sc, -msub));
+        for (int e = 0; e < 32; ++e) {
+          const int i = half * 64 + 2 * e;
+          const float p0 = ex2_approx(fmaf(s[i], sc, -msub));
+          const float p1 = ex2_approx(fmaf(s[i + 1], sc, -msub));
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           lsum += __low2float(pr) + __high2float(pr);
-          w4[e] = *reinterpret_cast<const uint32_t *>(&pr);
+          w[e] = __uint_as_float(*reinterpret_cast<const uint32_t *>(&pr));
         }
-        const int blk = c >> 3, cc = c & 7;
-        unsigned char *dst = sP + blk * K::BLK + (row >> 3) * 1024 + (row & 7) * 128 +
-                             ((cc ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        tc::tmem_st32(tmem + lane_base + K::TM_P + half * 32, w);
       }
+      tc::tmem_wait_st();
       l_run += lsum;
       if (kb + kBN > n_keys) {
         // Cells past the sequence in this V tile are not the sequence's (an
