@@ -1,20 +1,23 @@
 """Benchmark of the GQA hot path on B200 (one JSON line on rank 0).
 
 A step is one pass of the decode hot path over one batch: reset the lengths
-to the cached count, append the new token's K/V to the cache
-(gqa_cache_append), then decode it against the cache (gqa_decode: head map,
-permitted window, scores, online softmax, value mix, split-K merge).
-The default workload is bf16 decode with B=8, Hq=32, Hkv=8, d=128 and 8000
-cached cells per sequence (8001 keys read with the new token).
+to the cached count, then one gqa_decode_append call, which appends the new
+token's K/V row to the cache and decodes it against the cache in the same
+kernel (head map, permitted window, scores, online softmax, value mix,
+split-K merge).  The same step unfused (gqa_cache_append, then gqa_decode)
+is reported beside it.  The default workload is bf16 decode with B=8, Hq=32,
+Hkv=8, d=128 and 8000 cached cells per sequence (8001 keys read with the
+new token).
 
 value  = algorithmic bytes per step x steps x ranks / max-over-ranks time,
          algorithmic bytes = K+V of every permitted cell + Q + O + the
          appended rows (read and written)
-e2e    = the same through the public API with host buffers: pinned host->
-         device copies of q and the new K/V, and the device->host read of o,
-         inside the timed region
-roofline = the split-K decode (split + merge kernels) against the measured
-         HBM copy bandwidth
+e2e    = the same through the public API with host buffers: the pinned
+         host->device copy of the step's q and new K/V (one packed buffer)
+         and the device->host read of o inside the timed region; the step is
+         captured in a CUDA graph and replayed (the eager figure is beside it)
+roofline = the fused split-K decode kernel against the measured HBM copy
+         bandwidth
 cpu_baseline = the fp64 oracle on this host's cores on a bounded sample
 
 Usage: python bench.py [--gpus N --steps K --warmup W] [--impl reference]
@@ -206,10 +209,19 @@ class DecodeStep:
         self.C = C + extra
         B, Hq, d = w.B, w.Hq, w.d
         C = self.C
-        self.q, self.kc, self.vc = [t.to(device) for t in synthetic.decode_inputs(
-            B, Hq, self.Hkv, C, d, w.seed, std=w.std)]
-        self.kn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=21).to(device)
-        self.vn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=22).to(device)
+        q, kc, vc = synthetic.decode_inputs(B, Hq, self.Hkv, C, d, w.seed, std=w.std)
+        self.kc, self.vc = kc.to(device), vc.to(device)
+        kn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=21)
+        vn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=22)
+        # The step's inputs (q, k_new, v_new) are views of one buffer, so a
+        # single host->device copy brings a step's inputs in.
+        nq, nk = q.numel(), kn.numel()
+        self.inbuf = torch.empty(nq + 2 * nk, dtype=q.dtype, device=device)
+        self.q = self.inbuf[:nq].view(q.shape)
+        self.kn = self.inbuf[nq:nq + nk].view(kn.shape)
+        self.vn = self.inbuf[nq + nk:].view(vn.shape)
+        for dst, src in ((self.q, q), (self.kn, kn), (self.vn, vn)):
+            dst.copy_(src)
         self.lens0 = torch.tensor(self.cached, dtype=torch.int32, device=device)
         self.lens = self.lens0.clone()
         self.o = torch.empty_like(self.q)
@@ -253,11 +265,11 @@ class DecodeStep:
         self.gqa.decode(self.q, self.kc, self.vc, self.lens, window=self.window, out=self.o,
                         workspace=self.ws, status=self.status)
 
-    def run_host(self, hq, hkn, hvn, ho):
-        """One step through the public API from pinned host buffers."""
-        self.q.copy_(hq, non_blocking=True)
-        self.kn.copy_(hkn, non_blocking=True)
-        self.vn.copy_(hvn, non_blocking=True)
+    def run_host(self, hin, ho):
+        """One step through the public API: the step's inputs from a pinned
+        host buffer (q, k_new, v_new packed), the output back to pinned host
+        memory."""
+        self.inbuf.copy_(hin, non_blocking=True)
         self.run()
         ho.copy_(self.o, non_blocking=True)
 
@@ -483,26 +495,39 @@ def run_gpu(args, world, rank, local):
     total_ms = dist_max(total_ms, device)
     dec_avg_ms = sum(dec_ms) / K2
 
-    # end to end through the public API with pinned host buffers
-    hq = step.q.cpu().pin_memory()
-    hkn = step.kn.cpu().pin_memory()
-    hvn = step.vn.cpu().pin_memory()
+    # End to end through the public API with pinned host buffers: the step
+    # (host->device copy of the inputs, the fused call, device->host copy of
+    # the output) captured once in a CUDA graph and replayed per step, as a
+    # serving loop runs it; and the same step issued eagerly from Python.
+    hin = step.inbuf.cpu().pin_memory()
     ho = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
     for _ in range(2):
-        step.run_host(hq, hkn, hvn, ho)
+        step.run_host(hin, ho)
     torch.cuda.synchronize(device)
+    g_host = capture(lambda: step.run_host(hin, ho), device)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_ms = 0.0
+    e2e_ms = e2e_eager_ms = 0.0
     for i in range(K):
         if flush is not None:
             flush_l2(flush)
         e0.record(stream)
-        step.run_host(hq, hkn, hvn, ho)
+        g_host.replay()
         e1.record(stream)
         torch.cuda.synchronize(device)
         e2e_ms += e0.elapsed_time(e1)
+    for i in range(K):
+        if flush is not None:
+            flush_l2(flush)
+        e0.record(stream)
+        step.run_host(hin, ho)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_eager_ms += e0.elapsed_time(e1)
     e2e_ms = dist_max(e2e_ms, device)
+    e2e_eager_ms = dist_max(e2e_eager_ms, device)
+    if not torch.equal(ho.to(device), step.o):
+        raise RuntimeError("the output read back to the host differs from the device output")
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after timing")
 
@@ -514,7 +539,7 @@ def run_gpu(args, world, rank, local):
     peaks, peak_kind = measured_peaks()
     value = aggregate_rate(step.step_bytes, K, world, total_ms) / 1e9
     achieved = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
-    h2d = hq.numel() * hq.element_size() + hkn.numel() * hkn.element_size() * 2
+    h2d = hin.numel() * hin.element_size()
     d2h = ho.numel() * ho.element_size()
     line = None
     if rank == 0:
@@ -544,7 +569,12 @@ def run_gpu(args, world, rank, local):
                          "traffic": args.traffic if args.traffic is not None else
                          captured_traffic(w.name, "decode", args.window, args.hkv)},
             "e2e": {"value": round(aggregate_rate(step.step_bytes, K, world, e2e_ms) / 1e9, 2),
-                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "mode": "CUDA graph of the public-API step (pinned host->device copy of "
+                            "q/k_new/v_new, gqa_decode_append, device->host copy of o), "
+                            "replayed once per step",
+                    "eager": round(aggregate_rate(step.step_bytes, K, world, e2e_eager_ms) / 1e9, 2),
+                    "eager_mode": "the same step issued from Python each step"},
             "gpu_launches": step.launches_per_step * K,
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
