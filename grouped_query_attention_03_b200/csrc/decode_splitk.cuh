@@ -375,11 +375,14 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 
 // The last CTA to finish lane L merges its np partials (slots L+c0 ..):
 // m = max m_i, l = sum e^{m_i - m} l_i, o = sum e^{m_i - m} acc_i / l.
-// Each of the NT threads (t = 0 .. NT-1) owns QPT float4 groups of the lane's R x D output and
-// folds the partials in batches of NB with a running maximum, so the loads
-// of one batch (the partials' (m, l) pairs and accumulator groups, just
-// written by other CTAs and read through L2) are in flight together and a
-// lane of up to NB partials costs one round trip.
+// Each of the NT threads (t = 0 .. NT-1) owns QPT float4 groups of the
+// lane's R x D output.  The arithmetic does not depend on NT or on how the
+// loads are batched (a lane is merged by 224, 128 or 96 threads depending on
+// which CTA finishes it last, which is a matter of timing): m is the exact
+// maximum over all partials, then the terms are added in ascending i.  The
+// loads of the first NB partials and the maxima of the rest are issued
+// together, so a lane of up to NB partials costs one round trip through L2
+// (the partials were just written by other CTAs).
 template <int D, int R, int NT>
 __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
                                         __nv_bfloat16 *out, int rc, int t) {
@@ -389,42 +392,67 @@ __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
   const float2 *ml = p.ml + (size_t)(L + c0) * R;
   const float4 *acc4 = reinterpret_cast<const float4 *>(p.acc + (size_t)(L + c0) * R * D);
 
-  float m[QPT], l[QPT], x[QPT][4];
+  int hq[QPT];
+  bool live[QPT];
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) {
+    const int q4 = t + i * NT;
+    live[i] = q4 < G4;
+    hq[i] = live[i] ? q4 / (D / 4) : 0;
+  }
+  // the first batch: (m, l) pairs and accumulator groups
+  float2 mv[QPT][NB];
+  float4 a[QPT][NB];
+#pragma unroll
+  for (int i = 0; i < QPT; ++i)
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      if (live[i] && j < np) {
+        mv[i][j] = __ldcg(ml + (size_t)j * R + hq[i]);
+        a[i][j] = __ldcg(acc4 + (size_t)j * G4 + t + i * NT);
+      } else {
+        mv[i][j] = make_float2(-INFINITY, 0.f);
+        a[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+  // m = max over every partial (exact in any order)
+  float m[QPT];
 #pragma unroll
   for (int i = 0; i < QPT; ++i) {
     m[i] = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NB; ++j) m[i] = fmaxf(m[i], mv[i][j].x);
+  }
+  for (int j0 = NB; j0 < np; j0 += NB) {
+#pragma unroll
+    for (int i = 0; i < QPT; ++i)
+#pragma unroll
+      for (int j = 0; j < NB; ++j)
+        if (live[i] && j0 + j < np) m[i] = fmaxf(m[i], __ldcg(&ml[(size_t)(j0 + j) * R + hq[i]].x));
+  }
+  float l[QPT], x[QPT][4];
+#pragma unroll
+  for (int i = 0; i < QPT; ++i) {
     l[i] = 0.f;
     x[i][0] = x[i][1] = x[i][2] = x[i][3] = 0.f;
   }
   for (int j0 = 0; j0 < np; j0 += NB) {
-    float2 mv[QPT][NB];
-    float4 a[QPT][NB];
+    if (j0 > 0) {
 #pragma unroll
-    for (int i = 0; i < QPT; ++i) {
-      const int q4 = t + i * NT;
-      const int h = q4 / (D / 4);
+      for (int i = 0; i < QPT; ++i)
 #pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        if (q4 < G4 && j0 + j < np) {
-          mv[i][j] = __ldcg(ml + (size_t)(j0 + j) * R + h);
-          a[i][j] = __ldcg(acc4 + (size_t)(j0 + j) * G4 + q4);
-        } else {
-          mv[i][j] = make_float2(-INFINITY, 0.f);
-          a[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < NB; ++j) {
+          if (live[i] && j0 + j < np) {
+            mv[i][j] = __ldcg(ml + (size_t)(j0 + j) * R + hq[i]);
+            a[i][j] = __ldcg(acc4 + (size_t)(j0 + j) * G4 + t + i * NT);
+          } else {
+            mv[i][j] = make_float2(-INFINITY, 0.f);
+            a[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
-      }
     }
 #pragma unroll
-    for (int i = 0; i < QPT; ++i) {
-      float mb = m[i];
-#pragma unroll
-      for (int j = 0; j < NB; ++j) mb = fmaxf(mb, mv[i][j].x);
-      if (mb > m[i]) {
-        const float sc = m[i] == -INFINITY ? 0.f : exp2f(m[i] - mb);
-        l[i] *= sc;
-        x[i][0] *= sc; x[i][1] *= sc; x[i][2] *= sc; x[i][3] *= sc;
-        m[i] = mb;
-      }
+    for (int i = 0; i < QPT; ++i)
 #pragma unroll
       for (int j = 0; j < NB; ++j) {
         const float e = mv[i][j].x == -INFINITY ? 0.f : exp2f(mv[i][j].x - m[i]);
@@ -434,13 +462,11 @@ __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
         x[i][2] += e * a[i][j].z;
         x[i][3] += e * a[i][j].w;
       }
-    }
   }
 #pragma unroll
   for (int i = 0; i < QPT; ++i) {
     const int q4 = t + i * NT;
-    const int h = q4 / (D / 4);
-    if (q4 < G4 && h < rc) {
+    if (live[i] && hq[i] < rc) {
       const float inv = 1.f / l[i];
       *reinterpret_cast<uint2 *>(out + q4 * 4) =
           make_uint2(pack_bf16(x[i][0] * inv, x[i][1] * inv), pack_bf16(x[i][2] * inv, x[i][3] * inv));

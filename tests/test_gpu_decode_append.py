@@ -144,3 +144,36 @@ def test_decode_append_steps_track_oracle(cuda_lib):
         assert_close(o, want, torch.bfloat16, f"step {step}")
     np.testing.assert_array_equal(f64(kd), k64)
     np.testing.assert_array_equal(f64(vd), v64)
+
+
+def test_decode_append_is_bitwise_reproducible(cuda_lib):
+    """The same calls from the same cache give the same bits.  Which CTA
+    finishes a lane last, and so merges it (alone, with 224 threads, or next
+    to a second lane, with 128 or 96), is a matter of timing; the merge's
+    arithmetic must not depend on it.  Ragged MQA lengths (64 sequences,
+    uniform in [1, 8192]) give many lanes split over two to five CTAs."""
+    B, Hq, Hkv, d, calls = 64, 8, 1, 128, 100
+    lens = (synthetic.lengths_uniform(B, 1, 8192, 3)).tolist()
+    C = max(lens) + calls + 1
+    _, kc, vc = synthetic.decode_inputs(B, Hq, Hkv, C, d, 3)
+    kd0, vd0 = kc.to(DEV), vc.to(DEV)
+    qs = synthetic.normal((calls, B, Hq, d), 4, 1.0, torch.bfloat16, offset=11).to(DEV)
+    kn = synthetic.normal((calls, B, Hkv, 1, d), 4, 1.0, torch.bfloat16, offset=14).to(DEV)
+    vn = synthetic.normal((calls, B, Hkv, 1, d), 4, 1.0, torch.bfloat16, offset=15).to(DEV)
+    runs = []
+    for _ in range(2):
+        kd, vd = kd0.clone(), vd0.clone()
+        lt = torch.tensor(lens, dtype=torch.int32, device=DEV)
+        st = cuda_lib.new_status(DEV)
+        ws = cuda_lib.decode_workspace(qs[0], kd)
+        outs = torch.empty_like(qs)
+        for i in range(calls):
+            cuda_lib.decode_append(qs[i], kd, vd, kn[i], vn[i], lt, out=outs[i], workspace=ws,
+                                   status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        runs.append((outs, kd, vd, lt))
+    (o1, k1, v1, l1), (o2, k2, v2, l2) = runs
+    assert torch.equal(l1, l2) and torch.equal(k1, k2) and torch.equal(v1, v2)
+    differ = [i for i in range(calls) if not torch.equal(o1[i], o2[i])]
+    assert differ == [], f"calls whose outputs differ between identical runs: {differ}"
