@@ -132,36 +132,70 @@ def dist_max(x, device):
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu
 # captures summarised in profiles/, keyed by (workload, phase).  Each holds
-# the SHA-256 of the kernel's source files at capture time: once a source
-# changes the figure no longer describes the kernel and is reported as null.
+# the SHA-256 of the kernel's source files at capture time, comments and
+# blank lines stripped: once the code changes the figure no longer describes
+# the kernel and is reported as null (a comment edit does not count).
 CAPTURED_TRAFFIC = {
     ("decode_b8_n8000", "decode"): {
         "bytes": 268_888_576, "window": None, "hkv": None,
         "sources": ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "1dfdc85bab1638e282fca0346301a313dd0a68d6dc49c2c8dcf9bc05660cdac8",
+        "sha256": "469e7abd4723ef10c25be45c3b3cbd9aa34bb86e61b8ae0969f0048e75fed2f6",
         "profile": "profiles/decode_split_kernel_b8_n8000.md"},
     ("swa_t32768", "prefill"): {
         "bytes": 692_894_976, "window": 4096, "hkv": None,
         "sources": ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "1c048c911b18fbbb614c0d38605bc0f0c4d62456b0cebb82bffc519eb39dd8cd",
+        "sha256": "8c21ff11fc3aa0eda24d66f6c45b5c1a8fec2dec9750684743198082896bf26a",
         "profile": "profiles/prefill_pair_kernel_swa_t32768.md"},
 }
 
 
-def captured_traffic(workload, phase, window, hkv):
-    """ncu DRAM bytes per launch for this workload if the kernel's sources
-    are the captured ones, else None."""
+def strip_comments(src):
+    """C++/CUDA source without comments and blank lines (string and character
+    literals kept): what the compiler turns into the kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
+def source_digest(texts):
+    """SHA-256 over the comment-stripped sources, in order."""
     import hashlib
+    h = hashlib.sha256()
+    for t in texts:
+        h.update(strip_comments(t).encode())
+    return h.hexdigest()
+
+
+def captured_traffic(workload, phase, window, hkv):
+    """ncu DRAM bytes per launch for this workload if the kernel's code (its
+    sources without comments) is the captured code, else None."""
     c = CAPTURED_TRAFFIC.get((workload, phase))
     if c is None or window != c["window"] or hkv != c["hkv"]:
         return None
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)),
                         "grouped_query_attention_03_b200", "csrc")
-    h = hashlib.sha256()
+    texts = []
     for f in c["sources"]:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
-    return c["bytes"] if h.hexdigest() == c["sha256"] else None
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            texts.append(fh.read())
+    return c["bytes"] if source_digest(texts) == c["sha256"] else None
 
 
 def aggregate_rate(units_per_step, steps, world, max_ms):

@@ -8,9 +8,12 @@
 // blocks with a running max and sum instead of a materialised score row).
 //
 // Decomposition ("stream-K" over cache rows): the eligible rows of all
-// lanes (b, g) are laid end to end, total = Hkv * sum_b len_b, and CTA c takes
-// the contiguous range [c*per, (c+1)*per).  Every CTA gets the same number of
-// rows whatever the length mix, every cached byte is read once, and a CTA
+// lanes (b, g) are laid end to end, each non-empty lane preceded by `pad`
+// virtual rows that carry no work (so a lane segment's fixed cost -- query
+// load, combine, partial -- is charged as rows), total = VL * sum_b (len_b +
+// pad), and CTA c takes the contiguous range [c*per, (c+1)*per).  Every CTA
+// gets the same share whatever the length mix, every cached byte is read
+// once, and a CTA
 // writes one partial (m, l, acc) per lane its range touches, into slot
 // lane + c (an injective map: along the staircase of (c, lane) pairs each
 // step raises c, lane or both).
@@ -36,7 +39,9 @@
 // directly; otherwise the combined (m, l, acc) goes to the workspace and is
 // counted when the CTA's range ends (a per-lane atomic counter, zeroed at the
 // start of every call); the last CTA to count a lane merges the lane's
-// partials and writes bf16 output.  No CTA ever waits for another.
+// partials (the exact maximum first, then the terms in ascending order, so
+// the bits do not depend on which CTA comes last) and writes bf16 output.
+// No CTA ever waits for another.
 #pragma once
 
 #include <cuda.h>
