@@ -140,8 +140,9 @@ gqa_status gqa_prefill_packed(gqa_dtype dtype, const void *q, const void *k,
  *   dev_status device int32 (required)
  * bf16 with d in {64, 128}: split-K flash-decode (TMA-fed shared memory
  * ring, group heads stacked as tensor-core tile rows); the last CTA to
- * finish a lane merges that lane's partials.  Other d and fp32 run on CUDA
- * cores.
+ * finish a lane merges that lane's partials in a fixed order, so the same
+ * inputs give the same bits whichever CTA that is.  Other d and fp32 run on
+ * CUDA cores.
  */
 gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
                       const void *v_cache, void *o, const int32_t *seq_lens,
