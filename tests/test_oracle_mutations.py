@@ -41,6 +41,9 @@ MUTATIONS = [
      "long dst = ((b * Hkv + g) * W + (pos + 1) % W) * d;"),
     ("ring_window_short", "long lo = n > W ? n - W : 0;", "long lo = n > W ? n - W + 1 : 0;"),
     ("ring_overwrite_order", "if (t_new - i > W) continue;", "if (i >= W) continue;"),
+    ("segment_window_min", "return seg_start > sat ? seg_start : sat;",
+     "return seg_start < sat ? seg_start : sat;"),
+    ("no_window_is_self_only", "if (w < 0) return seg_start;", "if (w < 0) return t;"),
 ]
 
 
