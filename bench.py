@@ -409,6 +409,38 @@ def oracle_decode_sample(step, max_seconds):
             "seconds": dt}
 
 
+def oracle_prefill_sample(step, max_seconds):
+    """Time the fp64 oracle on a bounded sample of the same prefill: the last
+    query rows of one KV group of sequence 0.  The oracle's multi-token
+    decode over the whole prompt computes exactly those rows of the prefill
+    (with a window they are its steady-state rows)."""
+    import oracle
+    cores = oracle.set_threads(0)
+    w = step.w
+    r, T, d = w.Hq // step.Hkv, w.T, w.d
+    q = step.q[:1, :r].float().cpu().double().numpy()
+    k = step.k[:1, :1].float().cpu().double().numpy()
+    v = step.v[:1, :1].float().cpu().double().numpy()
+    lens = np.array([T])
+
+    def rows(t_new):
+        oracle.decode_multi(q[:, :, T - t_new:], k, v, lens, window=step.window)
+
+    t0 = time.perf_counter()
+    rows(8)
+    per_row = max((time.perf_counter() - t0) / 8, 1e-6)
+    t_new = int(max(1, min(T, max_seconds / per_row)))
+    t0 = time.perf_counter()
+    rows(t_new)
+    dt = time.perf_counter() - t0
+    pos = np.arange(T - t_new, T)
+    keys = np.minimum(pos + 1, step.window) if step.window else pos + 1
+    flops = 4 * d * int(keys.sum()) * r
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"the last {t_new} of {T} query rows of one KV group ({r} heads) of "
+                      f"sequence 0 (fp64)", "seconds": dt}
+
+
 def make_flush(device):
     """A 256 MB buffer whose read evicts the 126 MB L2 with clean lines (a
     write-based flush would leave dirty lines whose write-back the next
@@ -631,8 +663,51 @@ def run_gpu_prefill(args, world, rank, local):
     ms = dist_max(res["ms"], device)
     peaks, kind = measured_peaks()
     value = aggregate_rate(step.flops, 1, world, ms) / 1e12
+
+    # End to end through the public API: q, k, v copied in from pinned host
+    # memory and o copied back, inside the timed region; the step captured
+    # as a CUDA graph and replayed, and the same step issued eagerly.
+    hq, hk, hv = (t.cpu().pin_memory() for t in (step.q, step.k, step.v))
+    ho = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+
+    def run_host():
+        step.q.copy_(hq, non_blocking=True)
+        step.k.copy_(hk, non_blocking=True)
+        step.v.copy_(hv, non_blocking=True)
+        step.run()
+        ho.copy_(step.o, non_blocking=True)
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(2):
+        run_host()
+    torch.cuda.synchronize(device)
+    g_host = capture(run_host, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = e2e_eager_ms = 0.0
+    K_e2e = min(args.steps, 20)  # each step moves the whole prompt over PCIe
+    for i in range(K_e2e):
+        e0.record(stream)
+        g_host.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms += e0.elapsed_time(e1)
+    for i in range(K_e2e):
+        e0.record(stream)
+        run_host()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_eager_ms += e0.elapsed_time(e1)
+    e2e_ms = dist_max(e2e_ms, device)
+    e2e_eager_ms = dist_max(e2e_eager_ms, device)
+    if not torch.equal(ho.to(device), step.o):
+        raise RuntimeError("the output read back to the host differs from the device output")
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
     if rank != 0:
         return None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_prefill_sample(step, args.cpu_seconds)
     return {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
@@ -645,9 +720,16 @@ def run_gpu_prefill(args, world, rank, local):
                      "frac": res["frac_of_measured"], "frac_of_spec_2250": res["frac_of_spec_2250"],
                      "flops_per_launch": step.flops, "avg_launch_us": round(res["ms"] * 1e3, 2),
                      "traffic": args.traffic if args.traffic is not None else
-                     captured_traffic(w.name, "prefill", window, None)},
+                     captured_traffic(w.name, "prefill", window, args.hkv)},
+        "e2e": {"value": round(aggregate_rate(step.flops, K_e2e, world, e2e_ms) / 1e12, 2),
+                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "mode": "CUDA graph of the public-API step (pinned host->device copies of q, k "
+                        "and v, gqa_prefill, device->host copy of o), replayed once per step",
+                "eager": round(aggregate_rate(step.flops, K_e2e, world, e2e_eager_ms) / 1e12, 2),
+                "eager_mode": "the same step issued from Python each step", "steps": K_e2e},
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
     }
 
 

@@ -41,3 +41,35 @@ def test_traffic_only_for_the_captured_configuration():
     assert bench.captured_traffic("decode_b8_n8000", "decode", 512, None) is None
     assert bench.captured_traffic("decode_b8_n8000", "decode", None, 1) is None
     assert bench.captured_traffic("no_such_workload", "decode", None, None) is None
+    # the prefill capture is of the GQA shape; an MHA run (--hkv 32) has none
+    assert bench.captured_traffic("swa_t32768", "prefill", 4096, 32) is None
+
+
+def test_prefill_cpu_sample_rows_are_prefill_rows():
+    """The prefill CPU baseline times the oracle's multi-token decode of the
+    last rows of one KV group over the whole prompt; those are the same rows
+    of the oracle's prefill, and the sample's FLOPs count their keys."""
+    import types
+
+    import numpy as np
+    import torch
+
+    import oracle
+    from grouped_query_attention_03_b200 import synthetic
+
+    B, Hq, Hkv, T, d, window = 1, 4, 2, 64, 8, 16
+    q, k, v = synthetic.qkv_prefill(B, Hq, Hkv, T, d, 7)
+    r, t_new = Hq // Hkv, 24
+    f64 = lambda t: t.float().double().numpy()
+    full = oracle.prefill(f64(q), f64(k), f64(v), window=window)
+    tail = oracle.decode_multi(f64(q[:1, :r, T - t_new:]), f64(k[:1, :1]), f64(v[:1, :1]),
+                               np.array([T]), window=window)
+    assert np.array_equal(tail, full[:1, :r, T - t_new:])
+    w = types.SimpleNamespace(Hq=Hq, T=T, d=d)
+    step = types.SimpleNamespace(w=w, Hkv=Hkv, window=window, q=q, k=k, v=v)
+    try:
+        res = bench.oracle_prefill_sample(step, 0.05)
+    finally:
+        oracle.set_threads(1)
+    assert res["kind"] == "oracle" and res["unit"] == "TFLOP/s" and res["value"] > 0
+    assert res["cores"] >= 1 and "query rows of one KV group" in res["sample"]
