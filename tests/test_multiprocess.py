@@ -49,7 +49,8 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_max_time_and_aggregate():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    # spawn, not fork: earlier tests may have started the oracle's threads
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     assert sorted(out.keys()) == [0, 1]
     for r in range(world):
