@@ -381,8 +381,9 @@ def measure_prefill(w, window, device, reps, warmup, Hkv=None):
         "l2": "inputs exceed L2" if flush is None else "L2 flushed between launches"}
 
 
-def oracle_decode_sample(step, max_seconds):
-    """Time the fp64 oracle on a bounded sample of the same decode step."""
+def oracle_decode_sample(step, max_seconds, single=True):
+    """Time the fp64 oracle on a bounded sample of the same decode step (on
+    all host cores, and with `single` also on one thread)."""
     import oracle
     cores = oracle.set_threads(0)
     B = step.w.B
@@ -404,9 +405,28 @@ def oracle_decode_sample(step, max_seconds):
     n = lens[:nb]
     eff = np.minimum(n, step.window) if step.window else n
     bytes_ = reps * (2 * step.Hkv * eff.sum() * step.w.d * 2 + 2 * nb * step.w.Hq * step.w.d * 2)
-    return {"value": bytes_ / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{reps} x decode of {nb}/{B} sequences (fp64, all permitted cells)",
-            "seconds": dt}
+    res = {"value": bytes_ / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+           "sample": f"{reps} x decode of {nb}/{B} sequences (fp64, all permitted cells)",
+           "seconds": dt}
+    if not single:
+        return res
+    # the same on one thread: sequence 0 repeated for a third of the budget
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.decode(q[:1], kc[:1], vc[:1], lens[:1], window=step.window)
+        one = max(time.perf_counter() - t0, 1e-4)
+        reps1 = max(1, int(max_seconds / 3 / one))
+        t0 = time.perf_counter()
+        for _ in range(reps1):
+            oracle.decode(q[:1], kc[:1], vc[:1], lens[:1], window=step.window)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(0)
+    bytes1 = reps1 * (2 * step.Hkv * eff[0] * step.w.d * 2 + 2 * step.w.Hq * step.w.d * 2)
+    res["single_thread"] = {"value": bytes1 / dt1 / 1e9, "unit": "GB/s", "cores": 1,
+                            "sample": f"{reps1} x decode of sequence 0", "seconds": dt1}
+    return res
 
 
 def oracle_prefill_sample(step, max_seconds):
@@ -436,9 +456,23 @@ def oracle_prefill_sample(step, max_seconds):
     pos = np.arange(T - t_new, T)
     keys = np.minimum(pos + 1, step.window) if step.window else pos + 1
     flops = 4 * d * int(keys.sum()) * r
+    # the same on one thread, for a third of the budget
+    oracle.set_threads(1)
+    try:
+        t1 = int(max(1, min(T, max_seconds / 3 / (per_row * cores))))
+        t0 = time.perf_counter()
+        rows(t1)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(0)
+    pos1 = np.arange(T - t1, T)
+    keys1 = np.minimum(pos1 + 1, step.window) if step.window else pos1 + 1
+    flops1 = 4 * d * int(keys1.sum()) * r
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"the last {t_new} of {T} query rows of one KV group ({r} heads) of "
-                      f"sequence 0 (fp64)", "seconds": dt}
+                      f"sequence 0 (fp64)", "seconds": dt,
+            "single_thread": {"value": flops1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                              "sample": f"the last {t1} rows, same group", "seconds": dt1}}
 
 
 def make_flush(device):
@@ -747,8 +781,8 @@ def run_reference(args, world, rank):
     step.q, step.kc, step.vc = synthetic.decode_inputs(B, Hq, step.Hkv, C, d, w.seed, std=w.std)
     budget = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        oracle_decode_sample(step, budget)
-    samples = [oracle_decode_sample(step, budget) for _ in range(args.steps)]
+        oracle_decode_sample(step, budget, single=False)
+    samples = [oracle_decode_sample(step, budget, single=False) for _ in range(args.steps)]
     secs = sum(s["seconds"] for s in samples)
     value = statistics.mean(s["value"] for s in samples)
     n = np.array(step.cached) + 1
