@@ -1,32 +1,39 @@
 """Benchmark of the GQA hot path on B200 (one JSON line on rank 0).
 
-A step is one pass of the decode hot path over one batch: reset the lengths
-to the cached count, then one gqa_decode_append call, which appends the new
-token's K/V row to the cache and decodes it against the cache in the same
-kernel (head map, permitted window, scores, online softmax, value mix,
-split-K merge).  The same step unfused (gqa_cache_append, then gqa_decode)
-is reported beside it.  The default workload is bf16 decode with B=8, Hq=32,
-Hkv=8, d=128 and 8000 cached cells per sequence (8001 keys read with the
-new token).
+A step is one pass of the decode hot path over one batch: one
+gqa_decode_append call, which appends the new token's K/V row to the cache
+and decodes it against the cache in the same kernel (head map, permitted
+window, scores, online softmax, value mix, split-K merge).  Every step reads
+the same cells: each step has its own copy of the cached lengths, set before
+the timed pass.  The same step unfused (gqa_cache_append, then gqa_decode)
+is reported beside it.  The default workload is bf16 decode with B=8,
+Hq=32, Hkv=8, d=128 and 8000 cached cells per sequence (8001 keys read with
+the new token).
 
 value  = algorithmic bytes per step x steps x ranks / max-over-ranks time,
          algorithmic bytes = K+V of every permitted cell + Q + O + the
-         appended rows (read and written)
+         appended rows (read and written); the K-step timed pass is repeated
+         (at least 30 times and half a second) and the median pass reported
 e2e    = the same through the public API with host buffers: the pinned
          host->device copy of the step's q and new K/V (one packed buffer)
          and the device->host read of o inside the timed region; the step is
          captured in a CUDA graph and replayed (the eager figure is beside it)
-roofline = the fused split-K decode kernel against the measured HBM copy
-         bandwidth
+roofline = the fused split-K decode kernel alone (back-to-back calls) against
+         the measured HBM copy bandwidth
+decode = the same measurements on the other decode workloads: the ragged
+         MQA and MHA endpoints (B=64, Hq=8, Hkv 1 / 8) and the long-context
+         sliding-window step (64 successive steps after a 32768-cell prompt)
+prefill = prefill TFLOP/s on the long-context and the T=1024 workloads
 cpu_baseline = the fp64 oracle on this host's cores on a bounded sample
 
 Usage: python bench.py [--gpus N --steps K --warmup W] [--impl reference]
-                       [--workload NAME]
+                       [--workload NAME] [--phase decode|prefill]
 Multi-GPU (torchrun): every rank runs its own independent batch (replicas,
 weak scaling; the path has no exchange step), timing is max over ranks.
 """
 import argparse
 import json
+import math
 import os
 import statistics
 import sys
@@ -43,7 +50,15 @@ from grouped_query_attention_03_b200 import synthetic, workloads  # noqa: E402
 
 METRIC = "decode KV-cache HBM GB/s (% of 8 TB/s); prefill TFLOP/s (% bf16 peak)"
 SPEC_HBM_GBS = 8000.0
+SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126e6
+# Inputs below this many bytes are flushed from L2 before every timed call:
+# at twice the L2 size a step's reads can no longer hit lines left by the
+# previous step.
+FLUSH_BELOW_BYTES = 2 * L2_BYTES
+MIN_PASSES = 30          # timed passes per measurement (median reported)
+MIN_PASS_SECONDS = 0.5   # ... and at least this much timed time (headline)
 
 
 def measured_peaks():
@@ -130,22 +145,40 @@ def dist_max(x, device):
     return float(t.item())
 
 
+def dist_max_list(xs, device):
+    """Element-wise maximum over ranks of equally long lists (each rank's
+    per-pass times: pass i of the job took as long as its slowest rank)."""
+    import torch.distributed as dist
+    if not dist.is_initialized():
+        return list(xs)
+    t = torch.tensor(list(xs), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def pass_stats(ms):
+    """Median, spread and count of per-pass times (ms)."""
+    s = sorted(ms)
+    q = lambda f: s[min(len(s) - 1, int(f * (len(s) - 1) + 0.5))]
+    return {"passes": len(s), "median_ms": statistics.median(s), "min_ms": s[0],
+            "p10_ms": q(0.1), "p90_ms": q(0.9), "max_ms": s[-1]}
+
+
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu
-# captures summarised in profiles/, keyed by (workload, phase).  Each holds
-# the SHA-256 of the kernel's source files at capture time, comments and
-# blank lines stripped: once the code changes the figure no longer describes
-# the kernel and is reported as null (a comment edit does not count).
+# captures (the committed summaries name the workload and the kernel), keyed
+# by (workload, phase).  Each holds the SHA-256 of the kernel's source files
+# at capture time, comments and blank lines stripped: once the code changes
+# the figure no longer describes the kernel and is reported as null (a
+# comment edit does not count).
 CAPTURED_TRAFFIC = {
     ("decode_b8_n8000", "decode"): {
         "bytes": 268_888_576, "window": None, "hkv": None,
         "sources": ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "469e7abd4723ef10c25be45c3b3cbd9aa34bb86e61b8ae0969f0048e75fed2f6",
-        "profile": "profiles/decode_split_kernel_b8_n8000.md"},
+        "sha256": "469e7abd4723ef10c25be45c3b3cbd9aa34bb86e61b8ae0969f0048e75fed2f6"},
     ("swa_t32768", "prefill"): {
         "bytes": 692_894_976, "window": 4096, "hkv": None,
         "sources": ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "8c21ff11fc3aa0eda24d66f6c45b5c1a8fec2dec9750684743198082896bf26a",
-        "profile": "profiles/prefill_pair_kernel_swa_t32768.md"},
+        "sha256": "8c21ff11fc3aa0eda24d66f6c45b5c1a8fec2dec9750684743198082896bf26a"},
 }
 
 
@@ -210,6 +243,13 @@ def barrier():
         dist.barrier()
 
 
+def n_passes(one_pass_ms, device, min_passes=MIN_PASSES, min_seconds=0.0, max_passes=3000):
+    """How many timed passes to run: at least `min_passes` and at least
+    `min_seconds` of timed work, the same number on every rank."""
+    n = max(min_passes, int(math.ceil(min_seconds * 1e3 / max(one_pass_ms, 1e-3))))
+    return int(dist_max(float(min(n, max_passes)), device))
+
+
 # --------------------------------------------------------------- workloads
 def decode_shape(w, window):
     """(window, cached cells per sequence, capacity) of a decode step.  The
@@ -224,27 +264,30 @@ def decode_shape(w, window):
 
 
 class DecodeStep:
-    """Append one token per sequence and decode it; the lengths are reset to
-    the cached count first so every step reads the same number of cells.
+    """Append one token per sequence and decode it.
 
     The step is one gqa_decode_append call (the append fused into the decode
-    kernel); run_separate() is the same step as gqa_cache_append followed by
+    kernel) on a lengths buffer that holds the cached count; each timed step
+    gets its own such buffer (`lens_bufs`, set before the pass) so that every
+    step reads the same number of cells without a reset inside the timed
+    region.  run_separate() is the same step as gqa_cache_append followed by
     gqa_decode, reported beside it."""
 
-    def __init__(self, w, device, Hkv=None, window=None, extra=0):
+    def __init__(self, w, device, Hkv=None, window=None, extra=0, nbufs=1):
         from grouped_query_attention_03_b200 import gqa
         self.gqa = gqa
         self.w = w
         self.Hkv = Hkv or w.Hkv
         self.window, self.cached, C = decode_shape(w, window)
-        # `extra` spare cells of capacity let the fused call run back to back
-        # (each call appends one cell) when it is timed alone
+        # `extra` spare cells of capacity let calls run back to back on one
+        # lengths buffer (each call appends one cell)
         self.extra = extra
         self.C = C + extra
         B, Hq, d = w.B, w.Hq, w.d
         C = self.C
         q, kc, vc = synthetic.decode_inputs(B, Hq, self.Hkv, C, d, w.seed, std=w.std)
         self.kc, self.vc = kc.to(device), vc.to(device)
+        del kc, vc
         kn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=21)
         vn = synthetic.normal((B, self.Hkv, 1, d), w.seed, w.std, offset=22)
         # The step's inputs (q, k_new, v_new) are views of one buffer, so a
@@ -257,7 +300,8 @@ class DecodeStep:
         for dst, src in ((self.q, q), (self.kn, kn), (self.vn, vn)):
             dst.copy_(src)
         self.lens0 = torch.tensor(self.cached, dtype=torch.int32, device=device)
-        self.lens = self.lens0.clone()
+        self.lens_bufs = self.lens0.repeat(max(1, nbufs), 1).contiguous()
+        self.lens = self.lens_bufs[0]
         self.o = torch.empty_like(self.q)
         self.ws = gqa.decode_workspace(self.q, self.kc)
         self.status = gqa.new_status(device)
@@ -268,12 +312,16 @@ class DecodeStep:
         self.write_bytes = int(2 * B * self.Hkv * d * e)
         self.decode_bytes = self.kv_bytes + self.qo_bytes
         self.step_bytes = self.decode_bytes + self.write_bytes
-        self.launches_per_step = 1  # the fused kernel (plus a lengths copy and a counter memset)
+        self.launches_per_step = 1  # the fused kernel
         self.launches_separate = 3  # append copy + commit, split kernel
+        self.need_flush = self.cache_bytes_touched() < FLUSH_BELOW_BYTES
+
+    def cache_bytes_touched(self):
+        return self.kv_bytes
 
     def kv_bytes_at(self, grown):
         """K+V bytes one step reads when `grown` cells were appended since the
-        lengths were reset (the window caps the cells read)."""
+        lengths were set (the window caps the cells read)."""
         n = np.array(self.cached) + 1 + grown
         eff = np.minimum(n, self.window) if self.window else n
         return int(2 * self.Hkv * eff.sum() * self.w.d * 2)
@@ -282,29 +330,26 @@ class DecodeStep:
         return self.kv_bytes_at(grown) + self.qo_bytes + self.write_bytes
 
     def reset(self):
-        self.lens.copy_(self.lens0, non_blocking=True)
+        self.lens_bufs.copy_(self.lens0.expand_as(self.lens_bufs), non_blocking=True)
 
-    def run_kernel(self):
-        self.gqa.decode_append(self.q, self.kc, self.vc, self.kn, self.vn, self.lens,
+    def call(self, i=0):
+        """One gqa_decode_append call on lengths buffer i."""
+        self.gqa.decode_append(self.q, self.kc, self.vc, self.kn, self.vn, self.lens_bufs[i],
                                window=self.window, out=self.o, workspace=self.ws,
                                status=self.status)
 
-    def run(self):
-        self.reset()
-        self.run_kernel()
-
-    def run_separate(self):
-        self.reset()
-        self.gqa.cache_append(self.kc, self.vc, self.kn, self.vn, self.lens, status=self.status)
-        self.gqa.decode(self.q, self.kc, self.vc, self.lens, window=self.window, out=self.o,
+    def run_separate(self, i=0):
+        lens = self.lens_bufs[i]
+        self.gqa.cache_append(self.kc, self.vc, self.kn, self.vn, lens, status=self.status)
+        self.gqa.decode(self.q, self.kc, self.vc, lens, window=self.window, out=self.o,
                         workspace=self.ws, status=self.status)
 
-    def run_host(self, hin, ho):
+    def run_host(self, hin, ho, i=0):
         """One step through the public API: the step's inputs from a pinned
         host buffer (q, k_new, v_new packed), the output back to pinned host
         memory."""
         self.inbuf.copy_(hin, non_blocking=True)
-        self.run()
+        self.call(i)
         ho.copy_(self.o, non_blocking=True)
 
     def describe(self):
@@ -312,14 +357,228 @@ class DecodeStep:
         d = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": self.Hkv, "d": w.d,
              "window": self.window, "capacity": self.C - self.extra,
              "keys_read_per_seq": "cached+1 (the appended token)",
-             "l2": "inputs exceed the 126 MB L2; no flush" if self.kv_bytes > 126e6
-             else "L2 flushed before every step by reading a 256 MB buffer (outside the timed interval)",
-             "timing": "CUDA graph of one step replayed K times; CUDA events on the launching stream"}
+             "l2": "L2 flushed before every step by reading a 256 MB buffer (outside the "
+                   "timed interval)" if self.need_flush else
+                   "inputs exceed twice the 126 MB L2; no flush"}
         if w.ragged:
             d["cached_lengths"] = f"uniform [{w.ragged[0]}, {w.ragged[1]}], seed {w.seed}"
         else:
-            d["cached"] = w.cached
+            d["cached"] = self.cached[0]
         return d
+
+
+def make_flush(device):
+    """A 256 MB buffer whose read evicts the 126 MB L2 with clean lines (a
+    write-based flush would leave dirty lines whose write-back the next
+    kernel would pay for)."""
+    return torch.ones(64 << 20, dtype=torch.float32, device=device)
+
+
+def flush_l2(buf):
+    return buf.sum()
+
+
+def capture(fn, device):
+    """Capture fn() into a CUDA graph (on a side stream, as torch requires)."""
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device)
+    s.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(s):
+        fn()
+        torch.cuda.synchronize(device)
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream(device).wait_stream(s)
+    torch.cuda.synchronize(device)
+    return g
+
+
+def timed_calls(fns, device, flush=None):
+    """Device time (ms) of running the callables in `fns` in order.  Without
+    a flush: one event pair around all of them, back to back.  With a flush:
+    L2 is flushed before each, outside its own event pair, and the times are
+    summed."""
+    stream = torch.cuda.current_stream(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    if flush is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for f in fns:
+            f()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        return a.elapsed_time(b)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in fns]
+    for f, (a, b) in zip(fns, evs):
+        flush_l2(flush)
+        a.record(stream)
+        f()
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    return sum(a.elapsed_time(b) for a, b in evs)
+
+
+def repeat_passes(one_pass, device, min_passes=MIN_PASSES, min_seconds=0.0):
+    """Per-pass times (ms, max over ranks pass by pass) of `one_pass`."""
+    first = one_pass()
+    n = n_passes(first, device, min_passes, min_seconds)
+    ms = [first] + [one_pass() for _ in range(n - 1)]
+    return dist_max_list(ms, device)
+
+
+def measure_decode(w, device, args, world, Hkv=None, window=None, loop=None,
+                   separate=False, min_seconds=0.0, cpu_seconds=None, gpu_index=0):
+    """Time the fused decode step on one workload; returns (step, result).
+
+    steps   K steps, each gqa_decode_append on its own lengths buffer holding
+            the cached count (all set before the pass), so every step reads
+            the same cells.  Repeated passes; median reported.
+    kernel  gqa_decode_append alone, K2 calls in a row on one lengths buffer
+            from the cached count (call i reads i more cells, its bytes
+            counted so) -- with `loop` = K2 this is the workload's own loop
+            of successive decode steps.
+    e2e     the step through the public API with pinned host buffers.
+    """
+    K = args.steps
+    K2 = loop or min(K, 100)
+    nb = max(K, K2)
+    step = DecodeStep(w, device, Hkv=Hkv, window=window, extra=K2 + 2, nbufs=nb)
+    flush = make_flush(device) if step.need_flush else None
+    for i in range(args.warmup):
+        step.reset()
+        if flush is not None:
+            flush_l2(flush)
+        step.call(0)
+    torch.cuda.synchronize(device)
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} after warm-up")
+
+    # Each step / call captured once as a CUDA graph and replayed: the timed
+    # regions hold only device work (no per-call host overhead).
+    g_steps = [capture(lambda i=i: step.call(i), device) for i in range(K)]
+    g_call0 = g_steps[0] if K >= 1 else capture(lambda: step.call(0), device)
+    step.reset()
+
+    def steps_pass():
+        step.reset()
+        return timed_calls([g.replay for g in g_steps], device, flush)
+
+    def kernel_pass():
+        step.reset()
+        return timed_calls([g_call0.replay] * K2, device, flush)
+
+    # clocks sampled while the timed passes run
+    with ClockSampler(gpu_index) as clocks:
+        step_ms = repeat_passes(steps_pass, device, MIN_PASSES, min_seconds)
+        kern_ms = repeat_passes(kernel_pass, device, MIN_PASSES, min_seconds)
+    sep = None
+    if separate:
+        g_sep = [capture(lambda i=i: step.run_separate(i), device) for i in range(K)]
+
+        def sep_pass():
+            step.reset()
+            return timed_calls([g.replay for g in g_sep], device, flush)
+        sep_ms = repeat_passes(sep_pass, device)
+        sep = {"what": "gqa_cache_append then gqa_decode (same step, not fused)",
+               "value": round(aggregate_rate(step.step_bytes, K, world,
+                                             statistics.median(sep_ms)) / 1e9, 2),
+               "ms_per_step": round(statistics.median(sep_ms) / K, 5),
+               "gpu_launches_per_step": step.launches_separate}
+        del g_sep
+    step.reset()
+    torch.cuda.synchronize(device)
+
+    # End to end through the public API with pinned host buffers: the step
+    # (host->device copy of the inputs, the fused call, device->host copy of
+    # the output) captured once in a CUDA graph per lengths buffer and
+    # replayed, as a serving loop runs it; and the same step issued eagerly.
+    hin = step.inbuf.cpu().pin_memory()
+    ho = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    step.run_host(hin, ho, 0)
+    torch.cuda.synchronize(device)
+    g_host = [capture(lambda i=i: step.run_host(hin, ho, i), device) for i in range(K)]
+    step.reset()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(device)
+    barrier()
+    e2e_ms = e2e_eager_ms = 0.0
+    for i in range(K):
+        if flush is not None:
+            flush_l2(flush)
+        e0.record(stream)
+        g_host[i].replay()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_ms += e0.elapsed_time(e1)
+    step.reset()
+    for i in range(K):
+        if flush is not None:
+            flush_l2(flush)
+        e0.record(stream)
+        step.run_host(hin, ho, i)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_eager_ms += e0.elapsed_time(e1)
+    e2e_ms = dist_max(e2e_ms, device)
+    e2e_eager_ms = dist_max(e2e_eager_ms, device)
+    if not torch.equal(ho.to(device), step.o):
+        raise RuntimeError("the output read back to the host differs from the device output")
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {int(step.status.item())} after timing")
+    del g_steps, g_host
+    step.reset()
+
+    peaks, peak_kind = measured_peaks()
+    st = pass_stats(step_ms)
+    kt = pass_stats(kern_ms)
+    kern_bytes = sum(step.step_bytes_at(i) for i in range(K2))
+    achieved = kern_bytes / (kt["median_ms"] / 1e3) / 1e9
+    value = aggregate_rate(step.step_bytes, K, world, st["median_ms"]) / 1e9
+    h2d = hin.numel() * hin.element_size()
+    d2h = ho.numel() * ho.element_size()
+    res = {
+        **step.describe(),
+        "value": round(value, 2), "unit": "GB/s",
+        "ms_per_step": round(st["median_ms"] / K, 5),
+        "frac_of_spec_8TBs": round(value / SPEC_HBM_GBS, 4),
+        "bytes_per_step": step.step_bytes,
+        "timing": {"steps_per_pass": K, **{k: (round(v, 5) if isinstance(v, float) else v)
+                                           for k, v in st.items()},
+                   "what": "K steps per pass (a CUDA graph per step, each on its own lengths "
+                           "buffer); CUDA events on the launching stream; median pass"},
+        "roofline": {"bound": "hbm",
+                     "kernel": "gqa_decode_append (dec::split_kernel: fused append, "
+                               "in-kernel merge)",
+                     "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
+                     "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "frac_of_spec_8TBs": round(achieved / SPEC_HBM_GBS, 4),
+                     "bytes_per_launch": round(kern_bytes / K2),
+                     "launches_per_pass": K2,
+                     "avg_launch_us": round(kt["median_ms"] / K2 * 1e3, 3),
+                     "passes": kt["passes"],
+                     "pass_ms": {k: round(v, 5) for k, v in kt.items() if k != "passes"},
+                     "calls": ("successive decode steps from the cached length (the "
+                               "workload's loop)" if loop else
+                               "back to back from the cached length"),
+                     "traffic": captured_traffic(w.name, "decode", window, Hkv)},
+        "e2e": {"value": round(aggregate_rate(step.step_bytes, K, world, e2e_ms) / 1e9, 2),
+                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "mode": "CUDA graph of the public-API step (pinned host->device copy of "
+                        "q/k_new/v_new, gqa_decode_append, device->host copy of o), "
+                        "replayed once per step",
+                "eager": round(aggregate_rate(step.step_bytes, K, world, e2e_eager_ms) / 1e9, 2),
+                "eager_mode": "the same step issued from Python each step"},
+        "gpu_launches_per_step": step.launches_per_step,
+        "clocks": clocks.summary(),
+    }
+    if sep is not None:
+        res["separate_step"] = sep
+    if cpu_seconds:
+        res["cpu_baseline"] = oracle_decode_sample(step, cpu_seconds, single=True)
+    return step, res
 
 
 class PrefillStep:
@@ -356,48 +615,56 @@ class PrefillStep:
 
 def measure_prefill(w, window, device, reps, warmup, Hkv=None):
     """Per-launch prefill time (CUDA events), L2 flushed between launches
-    when the inputs fit in L2."""
+    when the inputs fit in L2; the mean over `reps` launches."""
     step = PrefillStep(w, device, window, Hkv)
-    flush = make_flush(device) if step.in_bytes <= 126e6 else None
+    flush = make_flush(device) if step.in_bytes <= L2_BYTES else None
     for _ in range(warmup):
         step.run()
     graph = capture(step.run, device)
+    stream = torch.cuda.current_stream(device)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(reps)]
     for a, b in evs:
         if flush is not None:
             flush_l2(flush)
-        a.record()
+        a.record(stream)
         graph.replay()
-        b.record()
+        b.record(stream)
     torch.cuda.synchronize(device)
-    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    per = [a.elapsed_time(b) for a, b in evs]
+    ms = dist_max(statistics.mean(per), device)
     peaks, kind = measured_peaks()
     tflops = step.flops / (ms / 1e3) / 1e12
     return step, {
         **step.describe(), "kernel": step.kernel(), "tflops": round(tflops, 2), "ms": round(ms, 4),
+        "median_ms": round(statistics.median(per), 4), "launches": reps,
         "flops": step.flops, "frac_of_measured": round(tflops / peaks["bf16_tflops"], 4),
-        "peak_kind": f"{kind} bf16 matmul (burst)", "frac_of_spec_2250": round(tflops / 2250.0, 4),
+        "peak_kind": f"{kind} bf16 matmul (burst)",
+        "frac_of_spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4),
         "l2": "inputs exceed L2" if flush is None else "L2 flushed between launches"}
 
 
 def oracle_decode_sample(step, max_seconds, single=True):
     """Time the fp64 oracle on a bounded sample of the same decode step (on
-    all host cores, and with `single` also on one thread)."""
+    all host cores, and with `single` also on one thread).  Only the sampled
+    sequences are copied to the host."""
     import oracle
     cores = oracle.set_threads(0)
     B = step.w.B
-    nb = B
-    q = step.q.float().cpu().double().numpy()
-    kc = step.kc.float().cpu().double().numpy()
-    vc = step.vc.float().cpu().double().numpy()
     lens = np.array(step.cached) + 1
+
+    def host(nb):
+        return tuple(t[:nb].float().cpu().double().numpy() for t in (step.q, step.kc, step.vc))
+
     # one calibration call on a single sequence, then size the sample
+    q, kc, vc = host(1)
     t0 = time.perf_counter()
-    oracle.decode(q[:1], kc[:1], vc[:1], lens[:1], window=step.window)
+    oracle.decode(q, kc, vc, lens[:1], window=step.window)
     per_seq = max(time.perf_counter() - t0, 1e-4)
     nb = int(max(1, min(B, max_seconds / per_seq)))
     reps = max(1, int(max_seconds / (per_seq * nb)))
+    if nb > 1:
+        q, kc, vc = host(nb)
     t0 = time.perf_counter()
     for _ in range(reps):
         oracle.decode(q[:nb], kc[:nb], vc[:nb], lens[:nb], window=step.window)
@@ -475,30 +742,12 @@ def oracle_prefill_sample(step, max_seconds):
                               "sample": f"the last {t1} rows, same group", "seconds": dt1}}
 
 
-def make_flush(device):
-    """A 256 MB buffer whose read evicts the 126 MB L2 with clean lines (a
-    write-based flush would leave dirty lines whose write-back the next
-    kernel would pay for)."""
-    return torch.ones(64 << 20, dtype=torch.float32, device=device)
-
-
-def flush_l2(buf):
-    return buf.sum()
-
-
-def capture(fn, device):
-    """Capture fn() into a CUDA graph (on a side stream, as torch requires)."""
-    g = torch.cuda.CUDAGraph()
-    s = torch.cuda.Stream(device)
-    s.wait_stream(torch.cuda.current_stream(device))
-    with torch.cuda.stream(s):
-        fn()
-        torch.cuda.synchronize(device)
-        with torch.cuda.graph(g, stream=s):
-            fn()
-    torch.cuda.current_stream(device).wait_stream(s)
-    torch.cuda.synchronize(device)
-    return g
+# The other decode workloads on the default line: (workload, Hkv, loop).
+DECODE_ENTRIES = (
+    (workloads.DECODE_RAGGED, 1, None),     # MQA endpoint
+    (workloads.DECODE_RAGGED, 8, None),     # MHA endpoint
+    (workloads.SWA_T32768, None, 64),       # 64 successive steps after the prompt
+)
 
 
 def run_gpu(args, world, rank, local):
@@ -507,179 +756,65 @@ def run_gpu(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = workloads.BY_NAME[args.workload]
-    K2 = min(args.steps, 100)  # back-to-back calls of the fused kernel alone
-    step = DecodeStep(w, device, Hkv=args.hkv, window=args.window, extra=K2 + 2)
-    stream = torch.cuda.current_stream(device)
-    need_flush = step.kv_bytes <= 126e6
-    flush = make_flush(device) if need_flush else None
-    for _ in range(args.warmup):
-        if flush is not None:
-            flush_l2(flush)
-        step.run()
-    torch.cuda.synchronize(device)
-    if int(step.status.item()) != 0:
-        raise RuntimeError(f"device status {int(step.status.item())} after warm-up")
-    # The step (fused), the same step unfused, and the gqa_decode_append call
-    # alone, captured once and replayed: the timed regions hold only device
-    # work (no per-call host overhead).
-    g_step = capture(step.run, device)
-    g_sep = capture(step.run_separate, device)
-    g_reset = capture(step.reset, device)
-    step.reset()
-    g_dec = capture(step.run_kernel, device)
+    step, head = measure_decode(
+        w, device, args, world, Hkv=args.hkv, window=args.window,
+        loop=w.decode_steps or None, separate=True, min_seconds=MIN_PASS_SECONDS,
+        gpu_index=local)
+    if args.traffic is not None:
+        head["roofline"]["traffic"] = args.traffic
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_decode_sample(step, args.cpu_seconds)
+    del step
+    torch.cuda.empty_cache()
 
-    def events(n):
-        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(n)]
-
-    K = args.steps
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize(device)
-    with ClockSampler(local) as clocks:
-        if flush is None:
-            # inputs exceed L2: steps back to back
-            start.record(stream)
-            for i in range(K):
-                g_step.replay()
-            end.record(stream)
-            torch.cuda.synchronize(device)
-            total_ms = start.elapsed_time(end)
-            start.record(stream)
-            for i in range(K):
-                g_sep.replay()
-            end.record(stream)
-            torch.cuda.synchronize(device)
-            sep_ms = start.elapsed_time(end)
-        else:
-            # L2 flushed (outside the timed intervals) before every step
-            step_ev, sep_ev = events(K), events(K)
-            for i in range(K):
-                flush_l2(flush)
-                step_ev[i][0].record(stream)
-                g_step.replay()
-                step_ev[i][1].record(stream)
-            for i in range(K):
-                flush_l2(flush)
-                sep_ev[i][0].record(stream)
-                g_sep.replay()
-                sep_ev[i][1].record(stream)
-            torch.cuda.synchronize(device)
-            total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
-            sep_ms = sum(a.elapsed_time(b) for a, b in sep_ev)
-        # the gqa_decode_append call alone, K2 calls in a row from the reset
-        # lengths (call i reads i more cells; its bytes are counted so)
-        g_reset.replay()
-        if flush is None:
-            # inputs exceed L2: the calls back to back, one event pair
-            start.record(stream)
-            for i in range(K2):
-                g_dec.replay()
-            end.record(stream)
-            torch.cuda.synchronize(device)
-            dec_ms = [start.elapsed_time(end)]
-        else:
-            dec_ev = events(K2)
-            for i in range(K2):
-                flush_l2(flush)
-                dec_ev[i][0].record(stream)
-                g_dec.replay()
-                dec_ev[i][1].record(stream)
-            torch.cuda.synchronize(device)
-            dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
-        g_reset.replay()
-        torch.cuda.synchronize(device)
-    dec_bytes = [step.step_bytes_at(i) for i in range(K2)]
-    barrier()
-    sep_ms = dist_max(sep_ms, device)
-    total_ms = dist_max(total_ms, device)
-    dec_avg_ms = sum(dec_ms) / K2
-
-    # End to end through the public API with pinned host buffers: the step
-    # (host->device copy of the inputs, the fused call, device->host copy of
-    # the output) captured once in a CUDA graph and replayed per step, as a
-    # serving loop runs it; and the same step issued eagerly from Python.
-    hin = step.inbuf.cpu().pin_memory()
-    ho = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
-    for _ in range(2):
-        step.run_host(hin, ho)
-    torch.cuda.synchronize(device)
-    g_host = capture(lambda: step.run_host(hin, ho), device)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_ms = e2e_eager_ms = 0.0
-    for i in range(K):
-        if flush is not None:
-            flush_l2(flush)
-        e0.record(stream)
-        g_host.replay()
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        e2e_ms += e0.elapsed_time(e1)
-    for i in range(K):
-        if flush is not None:
-            flush_l2(flush)
-        e0.record(stream)
-        step.run_host(hin, ho)
-        e1.record(stream)
-        torch.cuda.synchronize(device)
-        e2e_eager_ms += e0.elapsed_time(e1)
-    e2e_ms = dist_max(e2e_ms, device)
-    e2e_eager_ms = dist_max(e2e_eager_ms, device)
-    if not torch.equal(ho.to(device), step.o):
-        raise RuntimeError("the output read back to the host differs from the device output")
-    if int(step.status.item()) != 0:
-        raise RuntimeError(f"device status {int(step.status.item())} after timing")
+    decode_extra = None
+    if not args.no_extra:
+        decode_extra = []
+        for ew, hkv, loop in DECODE_ENTRIES:
+            if ew.name == w.name and hkv == args.hkv:
+                continue
+            s2, r2 = measure_decode(
+                ew, device, args, world, Hkv=hkv, loop=loop, gpu_index=local,
+                cpu_seconds=(args.cpu_seconds / 3 if rank == 0 and world == 1
+                             and not args.no_cpu_baseline else None))
+            decode_extra.append(r2)
+            del s2
+            torch.cuda.empty_cache()
 
     prefill_extra = None
-    if rank == 0 and not args.no_prefill:
-        prefill_extra = [measure_prefill(workloads.SWA_T32768, 4096, device, 10, 3)[1],
-                         measure_prefill(workloads.PREFILL_B4_T1024, None, device, 20, 3)[1],
-                         measure_prefill(workloads.PREFILL_B4_T1024, 256, device, 20, 3)[1]]
-    peaks, peak_kind = measured_peaks()
-    value = aggregate_rate(step.step_bytes, K, world, total_ms) / 1e9
-    achieved = sum(dec_bytes) / (sum(dec_ms) / 1e3) / 1e9
-    h2d = hin.numel() * hin.element_size()
-    d2h = ho.numel() * ho.element_size()
-    line = None
-    if rank == 0:
-        cpu = None
-        if world == 1 and not args.no_cpu_baseline:
-            cpu = oracle_decode_sample(step, args.cpu_seconds)
-        line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-            "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic (seeded N(0,1) rounded to bf16)",
-            "config": dict(step.describe(), parallelism=f"replicas x{world}"),
-            "frac_of_spec_8TBs": round(value / SPEC_HBM_GBS, 4),
-            "separate_step": {"what": "gqa_cache_append then gqa_decode (same step, not fused)",
-                              "value": round(aggregate_rate(step.step_bytes, K, world, sep_ms) / 1e9, 2),
-                              "ms_per_step": round(sep_ms / K, 5),
-                              "gpu_launches_per_step": step.launches_separate},
-            "roofline": {"bound": "hbm",
-                         "kernel": "gqa_decode_append (counter memset + dec::split_kernel: fused append, in-kernel merge)",
-                         "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
-                         "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
-                         "frac": round(achieved / peaks["hbm_gbs"], 4),
-                         "frac_of_spec_8TBs": round(achieved / SPEC_HBM_GBS, 4),
-                         "bytes_per_launch": round(statistics.mean(dec_bytes)),
-                         "launches_timed": K2,
-                         "avg_launch_us": round(dec_avg_ms * 1e3, 3),
-                         "traffic": args.traffic if args.traffic is not None else
-                         captured_traffic(w.name, "decode", args.window, args.hkv)},
-            "e2e": {"value": round(aggregate_rate(step.step_bytes, K, world, e2e_ms) / 1e9, 2),
-                    "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "mode": "CUDA graph of the public-API step (pinned host->device copy of "
-                            "q/k_new/v_new, gqa_decode_append, device->host copy of o), "
-                            "replayed once per step",
-                    "eager": round(aggregate_rate(step.step_bytes, K, world, e2e_eager_ms) / 1e9, 2),
-                    "eager_mode": "the same step issued from Python each step"},
-            "gpu_launches": step.launches_per_step * K,
-            "clocks": clocks.summary(),
-            "cpu_baseline": cpu,
-            "prefill": prefill_extra,
-        }
+    if not args.no_prefill:
+        prefill_extra = []
+        for pw, pwin, reps in ((workloads.SWA_T32768, 4096, 10),
+                               (workloads.PREFILL_B4_T1024, None, 50),
+                               (workloads.PREFILL_B4_T1024, 256, 50)):
+            prefill_extra.append(measure_prefill(pw, pwin, device, reps, 3)[1])
+            torch.cuda.empty_cache()
+
+    if rank != 0:
+        return None
+    timing = head.pop("timing")
+    line = {
+        "metric": METRIC, "value": head.pop("value"), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head.pop("ms_per_step"),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded N(0,1) rounded to bf16)",
+        "config": {**{k: head.pop(k) for k in ("workload", "B", "Hq", "Hkv", "d", "window",
+                                               "capacity", "keys_read_per_seq", "l2")},
+                   **({"cached": head.pop("cached")} if "cached" in head else {}),
+                   **({"cached_lengths": head.pop("cached_lengths")}
+                      if "cached_lengths" in head else {}),
+                   "timing": timing, "parallelism": f"replicas x{world}"},
+        "frac_of_spec_8TBs": head.pop("frac_of_spec_8TBs"),
+        "separate_step": head.pop("separate_step"),
+        "roofline": head.pop("roofline"),
+        "e2e": head.pop("e2e"),
+        "gpu_launches": head["gpu_launches_per_step"] * args.steps,
+        "clocks": head.pop("clocks"),
+        "cpu_baseline": cpu,
+        "decode": decode_extra,
+        "prefill": prefill_extra,
+    }
     return line
 
 
@@ -753,6 +888,7 @@ def run_gpu_prefill(args, world, rank, local):
                      "peak_kind": f"{kind} bf16 matmul (burst)", "unit": "TFLOP/s",
                      "frac": res["frac_of_measured"], "frac_of_spec_2250": res["frac_of_spec_2250"],
                      "flops_per_launch": step.flops, "avg_launch_us": round(res["ms"] * 1e3, 2),
+                     "median_launch_us": round(res["median_ms"] * 1e3, 2),
                      "traffic": args.traffic if args.traffic is not None else
                      captured_traffic(w.name, "prefill", window, args.hkv)},
         "e2e": {"value": round(aggregate_rate(step.flops, K_e2e, world, e2e_ms) / 1e12, 2),
@@ -804,8 +940,8 @@ def run_reference(args, world, rank):
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["own", "reference"], default="own")
     ap.add_argument("--workload", default=workloads.DECODE_B8_N8000.name)
     ap.add_argument("--hkv", type=int, default=None, help="override Hkv (ragged MQA/MHA endpoints)")
@@ -815,6 +951,8 @@ def parse_args(argv=None):
     ap.add_argument("--phase", choices=["decode", "prefill"], default="decode")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the prefill figures on the decode line")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other decode workloads on the decode line")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per launch for the roofline (default: the "
                          "captured figure while the kernel is unchanged, else null)")

@@ -72,16 +72,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and
-// sets *failed) if the wait ran past kWaitLimitNs or an earlier wait of the
-// same thread already failed.
+// sets *failed) if the wait ran past limit_ns (kWaitLimitNs in the kernels)
+// or an earlier wait of the same thread already failed.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          bool *failed) {
+                                          bool *failed,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (*failed) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *failed = true;
       return false;
     }
@@ -104,14 +105,15 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // Like mbar_wait, but polls without suspending: for short intra-CTA
 // barriers where a suspended warp would wake up late.
 __device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity,
-                                               bool *failed) {
+                                               bool *failed,
+                                               uint64_t limit_ns = kWaitLimitNs) {
   if (*failed) return false;
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (mbar_test_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *failed = true;
       return false;
     }

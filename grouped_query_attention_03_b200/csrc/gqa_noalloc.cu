@@ -21,9 +21,14 @@
 //     calls whose kernels overlap on the GPU (different streams, no ordering
 //     between them) race on the array and give wrong results.  Order them.
 //   - The first call on each device looks up the array's device address
-//     (cudaGetSymbolAddress with that device current) and caches it; make
-//     that first call before any stream capture begins.
+//     (cudaGetSymbolAddress with that device current) and caches it, keyed
+//     by the device's current context; make that first call before any
+//     stream capture begins.  After a cudaDeviceReset the device has a new
+//     context and the module is loaded again, so the next call looks the
+//     address up again (again: not inside a capture).
 //   - Nothing here calls cudaMalloc, cudaFree or an allocating library.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "../../include/gqa.h"
@@ -38,24 +43,62 @@ constexpr size_t kScratchBytes = GQA_NOALLOC_SCRATCH_BYTES;
 // be handed to a kernel.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
+// Unique id of the calling thread's current context (driver entry points
+// looked up through the runtime, so the library needs no libcuda link);
+// false if it cannot be read.
+bool current_context_id(unsigned long long *id) {
+  typedef CUresult (*GetCurrentFn)(CUcontext *);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr, *q = nullptr;
+    cudaDriverEntryPointQueryResult r1, r2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r1) ==
+            cudaSuccess &&
+        r1 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &q, cudaEnableDefault, &r2) ==
+            cudaSuccess &&
+        r2 == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+      get_id = reinterpret_cast<GetIdFn>(q);
+    } else {
+      cudaGetLastError();
+    }
+  });
+  CUcontext ctx = nullptr;
+  return get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+         get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 // Device address of the array on the current device, looked up once per
-// device.  Returns NULL (and leaves no CUDA error pending) on failure.
+// device and context (and on every call if the context id cannot be read).
+// Returns NULL (and leaves no CUDA error pending) on failure.
 void *scratch_on_current_device() {
   static std::mutex mu;
   static void *addr[64] = {};
+  static unsigned long long ctx_of[64] = {};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return nullptr;
   }
+  // With no current context yet (the caller has made no CUDA call on this
+  // thread) the id is unknown and the address is looked up, which makes the
+  // device's primary context current.
+  unsigned long long ctx = 0;
+  const bool have_ctx = current_context_id(&ctx);
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || !have_ctx || ctx_of[dev] != ctx) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
       cudaGetLastError();
+      addr[dev] = nullptr;
       return nullptr;
     }
     addr[dev] = p;
+    ctx_of[dev] = have_ctx ? ctx : 0;
   }
   return addr[dev];
 }

@@ -29,7 +29,7 @@ STATUS_NAMES = {
 EXPORTS = ("gqa_prefill", "gqa_prefill_packed", "gqa_decode", "gqa_decode_workspace_bytes",
            "gqa_decode_append", "gqa_decode_multi", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
            "gqa_ring_append", "gqa_ring_decode_append", "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
-           "gqa_version")
+           "gqa_version", "gqa_selftest_wait_timeout")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # GQA_NOALLOC_SCRATCH_BYTES in include/gqa.h
 
@@ -89,6 +89,8 @@ def _declare(L):
     L.gqa_status_string.restype = ctypes.c_char_p
     L.gqa_version.argtypes = []
     L.gqa_version.restype = ctypes.c_char_p
+    L.gqa_selftest_wait_timeout.argtypes = [i64, i32, vp, vp, vp]
+    L.gqa_selftest_wait_timeout.restype = i32
     return L
 
 
@@ -102,6 +104,14 @@ def _status_string(s):
 def _check(status, what):
     if status != 0:
         raise GQAError(status, what)
+
+
+def _run(dev, what, fn, *args):
+    """Call a C entry point with `dev` (the tensors' device) current: the
+    library looks up per-device state (SM count, fixed scratch address) on
+    the current device."""
+    with torch.cuda.device(dev):
+        _check(fn(*args), what)
 
 
 def _dtype_code(t):
@@ -147,11 +157,11 @@ def ring_append(k_ring, v_ring, k_new, v_new, seq_lens, *, status=None, stream=N
         raise ValueError("new K/V shape mismatch")
     dev = k_ring.device
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_ring_append(
-        _dtype_code(k_ring), _ptr(k_ring, "k_ring"), _ptr(v_ring, "v_ring", k_ring.dtype, dev),
-        _ptr(k_new, "k_new", k_ring.dtype, dev), _ptr(v_new, "v_new", k_ring.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hkv, W, d, t_new,
-        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_ring_append")
+    _run(dev, "gqa_ring_append", lib().gqa_ring_append,
+         _dtype_code(k_ring), _ptr(k_ring, "k_ring"), _ptr(v_ring, "v_ring", k_ring.dtype, dev),
+         _ptr(k_new, "k_new", k_ring.dtype, dev), _ptr(v_new, "v_new", k_ring.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hkv, W, d, t_new,
+         _ptr(st, "status", torch.int32, dev), _stream(stream, dev))
 
 
 def ring_decode_append(q, k_ring, v_ring, k_new, v_new, seq_lens, *, scale=None, out=None,
@@ -173,13 +183,13 @@ def ring_decode_append(q, k_ring, v_ring, k_new, v_new, seq_lens, *, scale=None,
     if workspace is None:
         workspace = decode_workspace(q, k_ring)
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_ring_decode_append(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k_ring, "k_ring", q.dtype, dev),
-        _ptr(v_ring, "v_ring", q.dtype, dev), _ptr(k_new, "k_new", q.dtype, dev),
-        _ptr(v_new, "v_new", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, W, d, float(scale),
-        _ptr(workspace, "workspace", torch.uint8, dev), workspace.numel(),
-        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_ring_decode_append")
+    _run(dev, "gqa_ring_decode_append", lib().gqa_ring_decode_append,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k_ring, "k_ring", q.dtype, dev),
+         _ptr(v_ring, "v_ring", q.dtype, dev), _ptr(k_new, "k_new", q.dtype, dev),
+         _ptr(v_new, "v_new", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, W, d, float(scale),
+         _ptr(workspace, "workspace", torch.uint8, dev), workspace.numel(),
+         _ptr(st, "status", torch.int32, dev), _stream(stream, dev))
     return out
 
 
@@ -201,11 +211,11 @@ def prefill(q, k, v, *, window=None, scale=None, seq_lens=None, out=None,
         out = torch.empty_like(q)
     dev = q.device
     st = status
-    _check(lib().gqa_prefill(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k, "k", q.dtype, dev), _ptr(v, "v", q.dtype, dev),
-        _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
-        B, Hq, Hkv, T, d, _window(window), float(scale),
-        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_prefill")
+    _run(dev, "gqa_prefill", lib().gqa_prefill,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k, "k", q.dtype, dev), _ptr(v, "v", q.dtype, dev),
+         _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
+         B, Hq, Hkv, T, d, _window(window), float(scale),
+         _ptr(st, "status", torch.int32, dev), _stream(stream, dev))
     return out
 
 
@@ -225,12 +235,12 @@ def prefill_packed(q, k, v, seg_start, *, window=None, scale=None, seq_lens=None
         out = torch.empty_like(q)
     dev = q.device
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_prefill_packed(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k, "k", q.dtype, dev), _ptr(v, "v", q.dtype, dev),
-        _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
-        _ptr(seg_start, "seg_start", torch.int32, dev),
-        B, Hq, Hkv, T, d, _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
-        _stream(stream, dev)), "gqa_prefill_packed")
+    _run(dev, "gqa_prefill_packed", lib().gqa_prefill_packed,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k, "k", q.dtype, dev), _ptr(v, "v", q.dtype, dev),
+         _ptr(out, "out", q.dtype, dev), _ptr(seq_lens, "seq_lens", torch.int32, dev),
+         _ptr(seg_start, "seg_start", torch.int32, dev),
+         B, Hq, Hkv, T, d, _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
+         _stream(stream, dev))
     return out
 
 
@@ -263,13 +273,12 @@ def decode(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,
     if workspace is None:
         workspace = decode_workspace(q, k_cache)
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_decode(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
-        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
-        _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
-        workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
-        "gqa_decode")
+    _run(dev, "gqa_decode", lib().gqa_decode,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+         _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
+         _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
+         workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev))
     return out
 
 
@@ -294,14 +303,13 @@ def decode_append(q, k_cache, v_cache, k_new, v_new, seq_lens, *, window=None, s
     if workspace is None:
         workspace = decode_workspace(q, k_cache)
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_decode_append(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
-        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(k_new, "k_new", q.dtype, dev),
-        _ptr(v_new, "v_new", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
-        _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
-        workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev)),
-        "gqa_decode_append")
+    _run(dev, "gqa_decode_append", lib().gqa_decode_append,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+         _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(k_new, "k_new", q.dtype, dev),
+         _ptr(v_new, "v_new", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
+         _window(window), float(scale), _ptr(workspace, "workspace", torch.uint8, dev),
+         workspace.numel(), _ptr(st, "status", torch.int32, dev), _stream(stream, dev))
     return out
 
 
@@ -320,12 +328,12 @@ def decode_multi(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=
         out = torch.empty_like(q)
     dev = q.device
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_decode_multi(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
-        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d, t_new,
-        _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
-        _stream(stream, dev)), "gqa_decode_multi")
+    _run(dev, "gqa_decode_multi", lib().gqa_decode_multi,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+         _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d, t_new,
+         _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
+         _stream(stream, dev))
     return out
 
 
@@ -344,12 +352,12 @@ def decode_noalloc(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, ou
         out = torch.empty_like(q)
     dev = q.device
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_decode_noalloc(
-        _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
-        _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
-        _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
-        _stream(stream, dev)), "gqa_decode_noalloc")
+    _run(dev, "gqa_decode_noalloc", lib().gqa_decode_noalloc,
+         _dtype_code(q), _ptr(q, "q"), _ptr(k_cache, "k_cache", q.dtype, dev),
+         _ptr(v_cache, "v_cache", q.dtype, dev), _ptr(out, "out", q.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hq, Hkv, C, d,
+         _window(window), float(scale), _ptr(st, "status", torch.int32, dev),
+         _stream(stream, dev))
     return out
 
 
@@ -362,11 +370,11 @@ def cache_append(k_cache, v_cache, k_new, v_new, seq_lens, *, status=None, strea
         raise ValueError("new K/V shape mismatch")
     dev = k_cache.device
     st = new_status(dev) if status is None else status
-    _check(lib().gqa_cache_append(
-        _dtype_code(k_cache), _ptr(k_cache, "k_cache"), _ptr(v_cache, "v_cache", k_cache.dtype, dev),
-        _ptr(k_new, "k_new", k_cache.dtype, dev), _ptr(v_new, "v_new", k_cache.dtype, dev),
-        _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hkv, C, d, t_new,
-        _ptr(st, "status", torch.int32, dev), _stream(stream, dev)), "gqa_cache_append")
+    _run(dev, "gqa_cache_append", lib().gqa_cache_append,
+         _dtype_code(k_cache), _ptr(k_cache, "k_cache"), _ptr(v_cache, "v_cache", k_cache.dtype, dev),
+         _ptr(k_new, "k_new", k_cache.dtype, dev), _ptr(v_new, "v_new", k_cache.dtype, dev),
+         _ptr(seq_lens, "seq_lens", torch.int32, dev), B, Hkv, C, d, t_new,
+         _ptr(st, "status", torch.int32, dev), _stream(stream, dev))
     return st
 
 
@@ -386,3 +394,17 @@ def window_start(t, window):
 
 def version():
     return lib().gqa_version().decode()
+
+
+def selftest_wait_timeout(limit_us, *, arrive=False, device=None, status=None, stream=None):
+    """Run the kernels' two bounded wait routines on mbarriers nobody
+    arrives on (arrive=False: both give up after limit_us and the kernel
+    records GQA_ERR_TIMEOUT) or that one thread completes first (arrive=True:
+    both succeed).  Returns (status, gave_up) device tensors."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    st = new_status(dev) if status is None else status
+    gave_up = torch.zeros(2, dtype=torch.int32, device=dev)
+    _run(dev, "gqa_selftest_wait_timeout", lib().gqa_selftest_wait_timeout,
+         int(limit_us), 1 if arrive else 0, _ptr(st, "status", torch.int32, dev),
+         _ptr(gave_up, "gave_up", torch.int32, dev), _stream(stream, dev))
+    return st, gave_up

@@ -277,8 +277,10 @@ gqa_status gqa_ring_decode_append(gqa_dtype dtype, const void *q, void *k_ring,
  *     kernels may overlap on the GPU (unordered streams) race on it: order
  *     them on one stream or with events.
  *   - The first call on each device looks up the array's address (with that
- *     device current) and caches it; make that first call before any stream
- *     capture begins.  A failed lookup returns GQA_ERR_CUDA.
+ *     device current) and caches it for the device's current context; make
+ *     that first call before any stream capture begins.  After a
+ *     cudaDeviceReset the next call looks it up again (also outside any
+ *     capture).  A failed lookup returns GQA_ERR_CUDA.
  */
 gqa_status gqa_decode_noalloc(gqa_dtype dtype, const void *q,
                               const void *k_cache, const void *v_cache,
@@ -319,6 +321,31 @@ int gqa_kv_head_for_query(int h, int Hq, int Hkv);
  * cell of query cell t, max(0, t - (w-1)) (0 for GQA_NO_WINDOW); -1 for an
  * invalid window or t < 0. */
 int gqa_window_start(int t, int window);
+
+/*
+ * gqa_selftest_wait_timeout -- exercises the kernels' bounded waits, for
+ * tests of the failure handling.  [P1] "Extend the existing full and cached
+ * attention paths": a failed operation reports an error and leaves nothing
+ * half done; here that means a kernel whose internal wait (an mbarrier
+ * phase that a copy, an MMA or other warps should complete) runs out of
+ * time records GQA_ERR_TIMEOUT and returns instead of hanging the GPU.
+ *
+ * Launches one CTA of two warps that run the library's two wait routines
+ * (suspending and polling) on mbarriers that no thread arrives on, each
+ * giving up after limit_us microseconds; no copy or MMA is in flight.
+ *   limit_us    1 .. 2,000,000 (else GQA_ERR_SHAPE)
+ *   arrive      nonzero: one thread completes both barriers first, so both
+ *               waits succeed (the control case)
+ *   dev_status  device int32: set to GQA_ERR_TIMEOUT when a wait gave up
+ *   gave_up     device int32 [2]: element w is incremented when warp w's
+ *               wait gave up (warp 0 suspending, warp 1 polling)
+ * Asynchronous on `stream`; the kernel runs for about limit_us when the
+ * waits run out.  Returns GQA_ERR_NULL for a NULL pointer and
+ * GQA_ERR_DEVICE off sm_100.
+ */
+gqa_status gqa_selftest_wait_timeout(int64_t limit_us, int arrive,
+                                     int32_t *dev_status, int32_t *gave_up,
+                                     gqa_stream_t stream);
 
 /* Static English text for a status code (never NULL). */
 const char *gqa_status_string(gqa_status status);

@@ -246,3 +246,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(gqa, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         gqa.lib()
+
+
+def test_selftest_wait_host_refusals(L):
+    """The wait self-test refuses a limit outside [1 us, 2 s] and NULL
+    pointers before any CUDA call (no GPU needed)."""
+    fake = ctypes.c_void_p(0x1000)
+    assert L.gqa_selftest_wait_timeout(0, 0, fake, fake, None) == SHAPE
+    assert L.gqa_selftest_wait_timeout(-5, 0, fake, fake, None) == SHAPE
+    assert L.gqa_selftest_wait_timeout(2000001, 0, fake, fake, None) == SHAPE
+    assert L.gqa_selftest_wait_timeout(1000, 0, None, fake, None) == NULL
+    assert L.gqa_selftest_wait_timeout(1000, 0, fake, None, None) == NULL

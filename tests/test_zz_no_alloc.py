@@ -7,17 +7,21 @@ cannot supply gqa_decode's workspace.  gqa_decode_noalloc runs the same
 kernels with the library's fixed device array as the workspace.  This test
 calls it through the C ABI (ctypes), twice in a row on different inputs so
 the second call starts from the first call's leftover scratch contents, and
-checks each result against gqa_decode with its own workspace, within the
-bf16 tolerance the parity tests use.  It also checks that sizes whose
+checks each result bit for bit against gqa_decode with its own workspace
+(the decode is reproducible bit for bit, so any stale scratch value that
+leaked into a result would show) and against the fp64 oracle within the
+bf16 tolerance of the parity tests.  It also checks that sizes whose
 workspace exceeds the fixed array are refused before any work is queued.
 
 The file is named so pytest collects it last.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from parity import assert_close, f64
 from grouped_query_attention_03_b200 import synthetic
 
@@ -39,7 +43,7 @@ def _noalloc(L, q, kc, vc, o, lens, window, status):
         ctypes.c_void_p(status.data_ptr()), stream)
 
 
-def test_noalloc_decode_matches_workspace_decode(cuda_lib):
+def test_noalloc_decode_matches_workspace_decode_and_oracle(cuda_lib):
     L = cuda_lib.lib()
     cases = [
         # 8 sequences x 32 query heads over 8 KV heads, 8001 keys each
@@ -48,17 +52,20 @@ def test_noalloc_decode_matches_workspace_decode(cuda_lib):
         dict(B=16, Hq=8, Hkv=1, C=3000, d=128,
              lens=synthetic.lengths_uniform(16, 0, 3000, 5).tolist(), window=700, seed=2),
     ]
+    torch.cuda.set_device(DEV)
     for c in cases:
-        q, kc, vc = (t.to(DEV) for t in synthetic.decode_inputs(
-            c["B"], c["Hq"], c["Hkv"], c["C"], c["d"], c["seed"]))
+        q, kc, vc = synthetic.decode_inputs(c["B"], c["Hq"], c["Hkv"], c["C"], c["d"], c["seed"])
+        qd, kd, vd = (t.to(DEV) for t in (q, kc, vc))
         lens = torch.tensor(c["lens"], dtype=torch.int32, device=DEV)
-        want = cuda_lib.decode(q, kc, vc, lens, window=c["window"])
+        want = cuda_lib.decode(qd, kd, vd, lens, window=c["window"])
         status = torch.zeros(1, dtype=torch.int32, device=DEV)
-        got = torch.full_like(q, float("nan"))
-        rc = _noalloc(L, q, kc, vc, got, lens, c["window"], status)
+        got = torch.full_like(qd, float("nan"))
+        rc = _noalloc(L, qd, kd, vd, got, lens, c["window"], status)
         torch.cuda.synchronize()
         assert rc == 0 and int(status.item()) == 0
-        assert_close(got, f64(want), torch.bfloat16, f"noalloc {c}")
+        assert torch.equal(got, want), f"noalloc differs from gqa_decode: {c}"
+        ref = oracle.decode(f64(q), f64(kc), f64(vc), np.array(c["lens"]), window=c["window"])
+        assert_close(got, ref, torch.bfloat16, f"noalloc vs oracle {c}")
 
 
 def test_noalloc_refuses_sizes_beyond_the_fixed_scratch(cuda_lib):
