@@ -455,10 +455,21 @@ def measure_decode(w, device, args, world, Hkv=None, window=None, loop=None,
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after warm-up")
 
-    # Each step / call captured once as a CUDA graph and replayed: the timed
-    # regions hold only device work (no per-call host overhead).
-    g_steps = [capture(lambda i=i: step.call(i), device) for i in range(K)]
-    g_call0 = g_steps[0] if K >= 1 else capture(lambda: step.call(0), device)
+    # The calls are captured as CUDA graphs and replayed, so the timed
+    # regions hold only device work (no per-call host overhead).  Back to
+    # back (no flush), one graph holds the whole pass, the way a serving
+    # loop replays its captured steps: each split kernel is a programmatic
+    # dependent of the one before.  With a flush between calls, one graph
+    # per call.
+    def graphs(fns):
+        if flush is None:
+            return [capture(lambda: [f() for f in fns], device)]
+        return [capture(f, device) for f in fns]
+
+    g_steps = graphs([lambda i=i: step.call(i) for i in range(K)])
+    step.reset()
+    g_kern = graphs([lambda: step.call(0)] * K2) if flush is None else \
+        [capture(lambda: step.call(0), device)] * K2
     step.reset()
 
     def steps_pass():
@@ -467,7 +478,7 @@ def measure_decode(w, device, args, world, Hkv=None, window=None, loop=None,
 
     def kernel_pass():
         step.reset()
-        return timed_calls([g_call0.replay] * K2, device, flush)
+        return timed_calls([g.replay for g in g_kern], device, flush)
 
     # clocks sampled while the timed passes run
     with ClockSampler(gpu_index) as clocks:
@@ -475,7 +486,7 @@ def measure_decode(w, device, args, world, Hkv=None, window=None, loop=None,
         kern_ms = repeat_passes(kernel_pass, device, MIN_PASSES, min_seconds)
     sep = None
     if separate:
-        g_sep = [capture(lambda i=i: step.run_separate(i), device) for i in range(K)]
+        g_sep = graphs([lambda i=i: step.run_separate(i) for i in range(K)])
 
         def sep_pass():
             step.reset()
@@ -527,7 +538,7 @@ def measure_decode(w, device, args, world, Hkv=None, window=None, loop=None,
         raise RuntimeError("the output read back to the host differs from the device output")
     if int(step.status.item()) != 0:
         raise RuntimeError(f"device status {int(step.status.item())} after timing")
-    del g_steps, g_host
+    del g_steps, g_kern, g_host
     step.reset()
 
     peaks, peak_kind = measured_peaks()
@@ -546,8 +557,11 @@ def measure_decode(w, device, args, world, Hkv=None, window=None, loop=None,
         "bytes_per_step": step.step_bytes,
         "timing": {"steps_per_pass": K, **{k: (round(v, 5) if isinstance(v, float) else v)
                                            for k, v in st.items()},
-                   "what": "K steps per pass (a CUDA graph per step, each on its own lengths "
-                           "buffer); CUDA events on the launching stream; median pass"},
+                   "what": ("K steps per pass, each on its own lengths buffer, replayed "
+                            "from one CUDA graph" if flush is None else
+                            "K steps per pass, each on its own lengths buffer, a CUDA graph "
+                            "per step with the L2 flush between them")
+                           + "; CUDA events on the launching stream; median pass"},
         "roofline": {"bound": "hbm",
                      "kernel": "gqa_decode_append (dec::split_kernel: fused append, "
                                "in-kernel merge)",

@@ -120,6 +120,19 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity,
   }
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Wait until the grids this one depends on (the previous kernel on the
+// stream, when launched with programmatic stream serialization) have
+// completed and their memory is visible; returns at once otherwise.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the dependent grid (the next kernel on the stream) to be scheduled;
+// its CTAs still wait in griddep_wait for this grid to complete.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------ bulk (TMA) copies
 // Non-tensor bulk copy global -> shared, completing on an mbarrier.  Both
 // addresses must be 16-byte aligned and `bytes` a multiple of 16.  No

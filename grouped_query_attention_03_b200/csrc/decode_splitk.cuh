@@ -37,11 +37,17 @@
 // At the end of a lane segment the warps' states are combined through the
 // just-consumed stage buffer.  A lane covered by one CTA is written out
 // directly; otherwise the combined (m, l, acc) goes to the workspace and is
-// counted when the CTA's range ends (a per-lane atomic counter, zeroed at the
-// start of every call); the last CTA to count a lane merges the lane's
-// partials (the exact maximum first, then the terms in ascending order, so
-// the bits do not depend on which CTA comes last) and writes bf16 output.
-// No CTA ever waits for another.
+// counted when the CTA's range ends (an atomic counter per split lane, kept
+// at the start of the workspace and indexed by the lane's first CTA); the
+// last CTA to count a lane resets the counter and merges the lane's partials
+// (the exact maximum first, then the terms in ascending order, so the bits
+// do not depend on which CTA comes last) and writes bf16 output.  Every
+// counter is zero when a call starts and zero again when it ends, so the
+// workspace needs no clearing between calls.  No CTA ever waits for another.
+//
+// Launched as a programmatic dependent of the previous kernel on the stream:
+// a CTA sets up its barriers while that kernel drains, then waits for it to
+// complete (griddepcontrol.wait) before its first access to global memory.
 #pragma once
 
 #include <cuda.h>
@@ -53,6 +59,11 @@ namespace gqa {
 namespace dec {
 
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
+// Largest grid; the workspace holds kMaxCtas split-lane counters (a split
+// lane's first CTA indexes it) and then the count of CTAs that have read
+// the lengths (fused append).
+constexpr int kMaxCtas = 1024;
+constexpr int kCtrFinish = kMaxCtas;
 // Lengths of up to this many sequences are cached in shared memory (read
 // from global memory once per CTA); a fused append needs that.
 constexpr int kLensSmem = 4096;
@@ -121,8 +132,11 @@ struct Params {
   int nsub;   // sub-groups of at most R heads per KV head
   int VL;     // virtual lanes per batch row = Hkv * nsub
   int min_rows;
-  int *counters;          // [B*VL + 1], zero at kernel start; the last
-                          // entry counts finished CTAs (fused append)
+  int *counters;          // [kMaxCtas + 1], zero at kernel start and left
+                          // zero: [c0] counts the partials of the split lane
+                          // whose first CTA is c0 (c0 is unique among split
+                          // lanes), [kCtrFinish] the CTAs that have read the
+                          // lengths (fused append)
   float2 *ml;             // [(grid + B*VL) * R]: (m, l)
   float *acc;             // [(grid + B*VL) * R * D]
   int32_t *status;
@@ -744,9 +758,13 @@ __device__ void consumer(const Params &p, unsigned char *smem,
     csync(comb, comb_count, &failed);
     if (threadIdx.x == 0) {
       fence_acq_rel_gpu();
-      const int o0 = atomicAdd(&p.counters[pL0], 1);
-      const int o1 = pend_n > 1 ? atomicAdd(&p.counters[pL1], 1) : 0;
+      const int o0 = atomicAdd(&p.counters[pc0], 1);
+      const int o1 = pend_n > 1 ? atomicAdd(&p.counters[pc1], 1) : 0;
       const int flags = (o0 == pn0 - 1 ? 1 : 0) | (pend_n > 1 && o1 == pn1 - 1 ? 2 : 0);
+      // The last count of a lane is its counter's last access in this call:
+      // leave it zero for the next call.
+      if (flags & 1) p.counters[pc0] = 0;
+      if (flags & 2) p.counters[pc1] = 0;
       if (flags) fence_acq_rel_gpu();
       merge_flag = flags;
     }
@@ -801,6 +819,13 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
     tc::prefetch_tmap(&tmV);
   }
   __syncthreads();
+  // Everything above touches only shared memory and the kernel parameters.
+  // From here on the CTA reads and writes global memory that the previous
+  // kernel on the stream may use: wait until it has completed (a no-op when
+  // the launch is not a programmatic dependent), then let the next kernel
+  // start its own set-up.
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == K::NWC) {
     producer<D, R>(p, &tmK, &tmV, smem, hdrs, full, empty, s_len, &s_bad, &lens_ready);
   } else {
@@ -819,8 +844,11 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
       int last = 0;
       if (lane == 0) {
         fence_acq_rel_gpu();
-        last = atomicAdd(&p.counters[p.B * p.VL], 1) == (int)gridDim.x - 1;
-        if (last) fence_acq_rel_gpu();
+        last = atomicAdd(&p.counters[kCtrFinish], 1) == (int)gridDim.x - 1;
+        if (last) {
+          p.counters[kCtrFinish] = 0;  // every CTA has counted: reset
+          fence_acq_rel_gpu();
+        }
       }
       last = __shfl_sync(0xffffffffu, last, 0);
       __syncwarp();

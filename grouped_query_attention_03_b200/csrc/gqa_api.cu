@@ -24,7 +24,7 @@ namespace {
 
 using bf16 = __nv_bfloat16;
 
-constexpr int kMaxDecodeCtas = 1024;  // workspace is sized for this many
+constexpr int kMaxDecodeCtas = gqa::dec::kMaxCtas;  // workspace is sized for this many
 #ifndef GQA_DEC_MIN_ROWS
 #define GQA_DEC_MIN_ROWS 256
 #endif
@@ -130,9 +130,10 @@ struct DecLayout {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace: per-lane arrival counters and one count of finished CTAs
-// (zeroed by each call), then the (m, l) and acc partials, one slot per
-// (lane, CTA) pair touching it.
+// Workspace: the arrival counters (one per possible first CTA of a split
+// lane, and one count of CTAs that have read the lengths) at a fixed place
+// for every shape, zero between calls; then the (m, l) and acc partials, one
+// slot per (lane, CTA) pair touching it.
 bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   const DecPlan pl = decode_plan(Hq, Hkv);
   int64_t lanes, slots, ml_elems, acc_elems;
@@ -142,7 +143,7 @@ bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   if (!elems(&acc_elems, {slots, pl.R, d})) return false;
   if (acc_elems > INT64_MAX / 8) return false;
   L->counters = 0;
-  L->counter_bytes = (size_t)(lanes + 1) * sizeof(int);
+  L->counter_bytes = (size_t)(gqa::dec::kCtrFinish + 1) * sizeof(int);
   L->ml = round256(L->counter_bytes);
   L->acc = L->ml + round256((size_t)ml_elems * sizeof(float2));
   L->total = L->acc + round256((size_t)acc_elems * sizeof(float));
@@ -180,7 +181,22 @@ gqa_status launch_splitk(const gqa::dec::Params &p, const void *k_cache,
   const int grid = std::min(kMaxDecodeCtas, K::MIN_BLOCKS * sms);
   // the lengths' shared-memory copy follows the stages
   const int smem = K::SMEM + (p.lens_smem ? ((p.B * 4 + 15) & ~15) : 0);
-  gqa::dec::split_kernel<D, R><<<grid, K::THREADS, smem, st>>>(mk, mv, p);
+  // A programmatic dependent of the previous kernel on the stream: its CTAs
+  // set up while that kernel drains and wait for it before touching memory.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(K::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gqa::dec::split_kernel<D, R>, mk, mv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -410,12 +426,14 @@ struct AppendArgs {
   int ring;  // the cache is a rolling buffer of C slots
 };
 
+// clear_counters: zero the workspace's counter region on the stream before
+// the split kernel (for a workspace the caller cannot clear itself).
 gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
                        const void *v_cache, void *o, const int32_t *seq_lens,
                        int B, int Hq, int Hkv, int C, int d, int window,
                        float scale, void *workspace, size_t workspace_bytes,
                        int32_t *dev_status, gqa_stream_t stream,
-                       const AppendArgs *ap) {
+                       const AppendArgs *ap, bool clear_counters = false) {
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
   if (B < 0 || C < 0) return GQA_ERR_SHAPE;
   gqa_status s = check_heads(Hq, Hkv, d);
@@ -476,7 +494,8 @@ gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
     p.lens_smem = B <= gqa::dec::kLensSmem ? 1 : 0;
     p.ring = (ap && ap->ring) ? 1 : 0;
     p.pad = kDecodeLanePadBytes / (4 * d);  // K and V rows of d bf16
-    if (cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
+    if (clear_counters &&
+        cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
       cudaGetLastError();
       return GQA_ERR_CUDA;
     }
@@ -515,6 +534,26 @@ gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
                      window, scale, workspace, workspace_bytes, dev_status,
                      stream, nullptr);
 }
+
+}  // extern "C"
+
+namespace gqa {
+namespace detail {
+gqa_status decode_clearing_counters(gqa_dtype dtype, const void *q,
+                                    const void *k_cache, const void *v_cache,
+                                    void *o, const int32_t *seq_lens, int B,
+                                    int Hq, int Hkv, int C, int d, int window,
+                                    float scale, void *workspace,
+                                    size_t workspace_bytes, int32_t *dev_status,
+                                    gqa_stream_t stream) {
+  return decode_impl(dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, C, d,
+                     window, scale, workspace, workspace_bytes, dev_status,
+                     stream, nullptr, true);
+}
+}  // namespace detail
+}  // namespace gqa
+
+extern "C" {
 
 gqa_status gqa_decode_append(gqa_dtype dtype, const void *q, void *k_cache,
                              void *v_cache, const void *k_new,

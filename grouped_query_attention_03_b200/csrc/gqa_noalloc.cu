@@ -16,10 +16,15 @@
 //   - Sizes whose workspace would not fit are rejected with
 //     GQA_ERR_WORKSPACE before anything is enqueued.
 //   - Every call on a device shares the one array, and it keeps whatever the
-//     last call wrote.  The decode kernels overwrite every workspace byte they
-//     read within the same call, so nothing has to start at zero; but two
-//     calls whose kernels overlap on the GPU (different streams, no ordering
-//     between them) race on the array and give wrong results.  Order them.
+//     last call wrote.  The decode kernels overwrite every partial they read
+//     within the same call; only the arrival counters at the start of the
+//     workspace must be zero when a kernel starts.  A call that completes
+//     leaves them zero, but one that gave up on a bounded wait may not, and
+//     a caller of this entry point cannot reach the array to clear it, so
+//     each call clears the counter region itself (a cudaMemsetAsync of a few
+//     KB on the caller's stream; no allocation).  Two calls whose kernels
+//     overlap on the GPU (different streams, no ordering between them) race
+//     on the array and give wrong results.  Order them.
 //   - The first call on each device looks up the array's device address
 //     (cudaGetSymbolAddress with that device current) and caches it, keyed
 //     by the device's current context; make that first call before any
@@ -33,6 +38,20 @@
 
 #include "../../include/gqa.h"
 #include "common.cuh"
+
+namespace gqa {
+namespace detail {
+// gqa_decode, clearing the workspace's counter region on the stream right
+// before the kernel (defined with the other entry points).
+gqa_status decode_clearing_counters(gqa_dtype dtype, const void *q,
+                                    const void *k_cache, const void *v_cache,
+                                    void *o, const int32_t *seq_lens, int B,
+                                    int Hq, int Hkv, int C, int d, int window,
+                                    float scale, void *workspace,
+                                    size_t workspace_bytes, int32_t *dev_status,
+                                    gqa_stream_t stream);
+}  // namespace detail
+}  // namespace gqa
 
 namespace {
 
@@ -117,6 +136,9 @@ extern "C" gqa_status gqa_decode_noalloc(gqa_dtype dtype, const void *q,
   if (need > kScratchBytes) return GQA_ERR_WORKSPACE;
   void *ws = scratch_on_current_device();
   if (!ws) return GQA_ERR_CUDA;
-  return gqa_decode(dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, C, d,
-                    window, scale, ws, kScratchBytes, dev_status, stream);
+  // gqa_decode's path, with the counter region cleared on the stream after
+  // every host-side check has passed and just before the kernel.
+  return gqa::detail::decode_clearing_counters(
+      dtype, q, k_cache, v_cache, o, seq_lens, B, Hq, Hkv, C, d, window, scale,
+      ws, kScratchBytes, dev_status, stream);
 }

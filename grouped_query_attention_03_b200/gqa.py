@@ -250,11 +250,13 @@ def decode_workspace_bytes(dtype, B, Hq, Hkv, C, d):
 
 
 def decode_workspace(q, k_cache):
-    """A device workspace large enough for decode on these shapes."""
+    """A zero-filled device workspace large enough for decode on these
+    shapes (reusable by later calls of any shape that fits)."""
     B, Hq, d = q.shape
     Hkv, C = k_cache.shape[1], k_cache.shape[2]
     n = decode_workspace_bytes(q.dtype, B, Hq, Hkv, C, d)
-    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    # zero-filled once; every completed call leaves it ready for the next
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=q.device)
 
 
 def decode(q, k_cache, v_cache, seq_lens, *, window=None, scale=None, out=None,

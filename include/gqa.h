@@ -135,14 +135,20 @@ gqa_status gqa_prefill_packed(gqa_dtype dtype, const void *q, const void *k,
  *   o        [B,Hq,d]      output
  *   seq_lens device int32 [B], each in [0, C]
  *   workspace / workspace_bytes  device scratch of at least
- *            gqa_decode_workspace_bytes(...) bytes, 256-byte aligned; its
- *            contents need no initialisation and are not preserved
+ *            gqa_decode_workspace_bytes(...) bytes, 256-byte aligned.  Fill
+ *            it with zeros once before its first use; every call that
+ *            completes leaves it ready for the next call of any shape, so it
+ *            needs no clearing between calls.  After a call that set
+ *            GQA_ERR_TIMEOUT, zero it again.  Calls sharing a workspace must
+ *            be ordered (one stream, or events).
  *   dev_status device int32 (required)
  * bf16 with d in {64, 128}: split-K flash-decode (TMA-fed shared memory
  * ring, group heads stacked as tensor-core tile rows); the last CTA to
  * finish a lane merges that lane's partials in a fixed order, so the same
- * inputs give the same bits whichever CTA that is.  Other d and fp32 run on
- * CUDA cores.
+ * inputs give the same bits whichever CTA that is.  That kernel is launched
+ * as a programmatic dependent of the previous kernel on the stream: its set
+ * up overlaps that kernel's tail, and it touches memory only after that
+ * kernel has completed.  Other d and fp32 run on CUDA cores.
  */
 gqa_status gqa_decode(gqa_dtype dtype, const void *q, const void *k_cache,
                       const void *v_cache, void *o, const int32_t *seq_lens,
@@ -273,9 +279,11 @@ gqa_status gqa_ring_decode_append(gqa_dtype dtype, const void *q, void *k_ring,
  *     GQA_NOALLOC_SCRATCH_BYTES return GQA_ERR_WORKSPACE; nothing is
  *     enqueued.  All other arguments and errors are those of gqa_decode.
  *   - All calls on a device share the one array, which keeps the last
- *     call's contents; nothing in it needs to start at zero.  Calls whose
- *     kernels may overlap on the GPU (unordered streams) race on it: order
- *     them on one stream or with events.
+ *     call's contents.  Each call first clears the part that must start at
+ *     zero (its few-KB counter region, one cudaMemsetAsync, no allocation);
+ *     the rest needs no initial value.  Calls whose kernels may overlap on
+ *     the GPU (unordered streams) race on it: order them on one stream or
+ *     with events.
  *   - The first call on each device looks up the array's address (with that
  *     device current) and caches it for the device's current context; make
  *     that first call before any stream capture begins.  After a

@@ -5,8 +5,11 @@ dec::producer (csrc/decode_splitk.cuh) lays the eligible rows of every
 rows, and CTA c takes [c*per, (c+1)*per).  This model walks the same way and
 checks what the kernel relies on: every real row is read by exactly one CTA,
 the (c0, np) a stage header carries are exactly the CTAs holding that lane
-(the merge counts arrivals against np), and the partial slot lane + CTA is
-never shared.  The GPU parity tests check the numbers; this checks the plan
+(the merge counts arrivals against np), the partial slot lane + CTA is
+never shared, and no two split lanes (np > 1) share a first CTA c0 (the
+arrival counter of a split lane is the workspace word indexed by c0), with
+c0 below the grid size, and no CTA holds more than two split lanes (its
+first and its last segment; the kernel keeps two pending counts).  The GPU parity tests check the numbers; this checks the plan
 over thousands of length mixes that the GPU tests cannot afford.
 """
 import random
@@ -77,6 +80,14 @@ def check(lens, VL, G, min_rows, pad):
     slots = [s[4] for s in segs]
     assert len(slots) == len(set(slots))
     assert max(s[0] for s in segs) < G
+    split = {L: c0 for c, L, c0, npc, _ in segs if npc > 1}
+    assert len(set(split.values())) == len(split), "two split lanes share a counter"
+    assert all(0 <= c0 < G for c0 in split.values())
+    per_cta = {}
+    for c, L, c0, npc, _ in segs:
+        if npc > 1:
+            per_cta.setdefault(c, set()).add(L)
+    assert all(len(v) <= 2 for v in per_cta.values())
 
 
 def test_split_plan_random_length_mixes():
