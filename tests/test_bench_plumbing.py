@@ -73,3 +73,21 @@ def test_prefill_cpu_sample_rows_are_prefill_rows():
         oracle.set_threads(1)
     assert res["kind"] == "oracle" and res["unit"] == "TFLOP/s" and res["value"] > 0
     assert res["cores"] >= 1 and "query rows of one KV group" in res["sample"]
+
+
+def test_pass_stats_median_and_spread():
+    st = bench.pass_stats([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert st["passes"] == 5 and st["median_ms"] == 3.0
+    assert st["min_ms"] == 1.0 and st["max_ms"] == 5.0
+    assert st["p10_ms"] == 1.0 and st["p90_ms"] == 5.0
+
+
+def test_pass_count_covers_minimum_passes_and_time():
+    import torch
+    cpu = torch.device("cpu")
+    # a 1 ms pass: 30 passes are 30 ms, so half a second needs 500
+    assert bench.n_passes(1.0, cpu, min_passes=30, min_seconds=0.5) == 500
+    # a 100 ms pass: the 30-pass minimum decides
+    assert bench.n_passes(100.0, cpu, min_passes=30, min_seconds=0.5) == 30
+    # never more than the cap
+    assert bench.n_passes(1e-6, cpu, min_passes=30, min_seconds=10.0) == 3000
