@@ -57,6 +57,14 @@ struct Warps {
                     kThreads * (SPLIT == 1 ? 168 : 96),
                 "register split exceeds the launch's registers");
 };
+// Pairs of every 8 whose exponentials the two-warpgroup softmax computes on
+// the FMA pipe (interior tiles only), per head width.
+#ifndef GQA_PF2_EMU64
+#define GQA_PF2_EMU64 0
+#endif
+#ifndef GQA_PF2_EMU128
+#define GQA_PF2_EMU128 0
+#endif
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 12;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -133,9 +141,12 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 // unit; masked cells give exactly 0), written as bf16 P into this thread's
 // TMEM lane over the S columns it came from (column c holds p[2c], p[2c+1]),
 // where the P V MMA reads it as its A operand; returns the row sum.
-// NS scores, stored CH (32 or 16) P columns at a time.
-template <int NS, int CH = 32>
-__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP) {
+// NS scores, stored CH (32 or 16) P columns at a time.  With `poly`, EMU
+// of every 8 pairs take the FMA-pipe exponential (cells that are all
+// permitted only: it does not flush -inf to an exact zero).
+template <int NS, int CH = 32, int EMU = 0>
+__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP,
+                                        bool poly = false) {
   float2 lsum2 = make_float2(0.f, 0.f);
   const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
 #pragma unroll
@@ -145,7 +156,9 @@ __device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint3
     for (int e = 0; e < CH; ++e) {
       const int i = part * 2 * CH + 2 * e;
       const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
-      const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      const float2 pv = (EMU > 0 && (e & 7) < EMU && poly)
+                            ? ex2_poly2(x)
+                            : make_float2(ex2_approx(x.x), ex2_approx(x.y));
       lsum2 = fadd2v(lsum2, pv);
       w[e] = __uint_as_float(pack_bf16(pv.x, pv.y));
     }
@@ -362,7 +375,8 @@ __device__ __forceinline__ void softmax_half(const Params &p, Bars &bars, float 
       l_run *= alpha;
       m_run = m_new;
     }
-    const float lsum = emit_p<NC, 16>(s, sc, m_run == -INFINITY ? 0.f : m_run, tP);
+    constexpr int EMU = D == 64 ? GQA_PF2_EMU64 : GQA_PF2_EMU128;
+    const float lsum = emit_p<NC, 16, EMU>(s, sc, m_run == -INFINITY ? 0.f : m_run, tP, !edge);
     l_run += lsum;
     tc::fence_before_sync();
     __syncwarp();
