@@ -32,8 +32,6 @@
 
 #include <cuda.h>
 
-#include <cstdlib>
-
 #include "common.cuh"
 #include "tc_ptx.cuh"
 #include "tma_host.cuh"
@@ -42,29 +40,11 @@ namespace gqa {
 namespace pf2 {
 
 constexpr int kBM = 128, kBN = 128;
-// SPLIT softmax warpgroups per head: 1 (each thread owns a whole 128-score
-// row) or 2 (two warpgroups share each row, 64 score columns each).
-template <int SPLIT>
-struct Warps {
-  static constexpr int kThreads = 128 + 2 * SPLIT * 128;
-  // Registers per thread after the split: the first warpgroup (producer,
-  // MMA issuer, two idle warps) gives registers to the softmax warpgroups.
-  // 128 * kRegsLow + (kThreads - 128) * kRegsHigh must not exceed
-  // kThreads * (launch registers): 384 x 168 for SPLIT 1, 640 x 96 for 2.
-  static constexpr int kRegsLow = SPLIT == 1 ? 72 : 56;
-  static constexpr int kRegsHigh = SPLIT == 1 ? 216 : 104;
-  static_assert(128 * kRegsLow + (kThreads - 128) * kRegsHigh <=
-                    kThreads * (SPLIT == 1 ? 168 : 96),
-                "register split exceeds the launch's registers");
-};
-// Pairs of every 8 whose exponentials the two-warpgroup softmax computes on
-// the FMA pipe (interior tiles only), per head width.
-#ifndef GQA_PF2_EMU64
-#define GQA_PF2_EMU64 0
-#endif
-#ifndef GQA_PF2_EMU128
-#define GQA_PF2_EMU128 0
-#endif
+constexpr int kThreads = 384;
+// Registers per thread after the split: the first warpgroup (producer, MMA
+// issuer, two idle warps) gives registers to the two softmax warpgroups.
+// 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * (launch registers).
+constexpr int kRegsLow = 72, kRegsHigh = 216;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 12;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -115,24 +95,22 @@ struct Bars {
   uint64_t q_full;
   uint64_t full[kMaxSlots], empty[kMaxSlots];
   uint64_t s_full[2], p_full[2], o_done[2];
-  uint64_t x_full[2];  // SPLIT 2: both halves of a head posted their value
   uint64_t mma_fin;
   uint64_t v_clean;  // the last V tile's rows past the sequence are zero
   uint32_t tmem_base;
 };
 
-// O *= alpha over NCOL columns of this thread's TMEM lane (the whole warp
-// takes part), CH (32 or 16) columns at a time.
-template <int NCOL, int CH = 32>
+// O *= alpha for this thread's TMEM lane (the whole warp takes part).
+template <int D>
 __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 #pragma unroll
-  for (int c = 0; c < NCOL / CH; ++c) {
-    float ov[CH];
-    if (CH == 32) tc::tmem_ld32(tO + c * CH, ov); else tc::tmem_ld16(tO + c * CH, ov);
+  for (int c = 0; c < D / 32; ++c) {
+    float ov[32];
+    tc::tmem_ld32(tO + c * 32, ov);
     tc::tmem_wait_ld();
 #pragma unroll
-    for (int i = 0; i < CH; ++i) ov[i] *= alpha;
-    if (CH == 32) tc::tmem_st32(tO + c * CH, ov); else tc::tmem_st16(tO + c * CH, ov);
+    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+    tc::tmem_st32(tO + c * 32, ov);
   }
   tc::tmem_wait_st();
 }
@@ -141,28 +119,22 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 // unit; masked cells give exactly 0), written as bf16 P into this thread's
 // TMEM lane over the S columns it came from (column c holds p[2c], p[2c+1]),
 // where the P V MMA reads it as its A operand; returns the row sum.
-// NS scores, stored CH (32 or 16) P columns at a time.  With `poly`, EMU
-// of every 8 pairs take the FMA-pipe exponential (cells that are all
-// permitted only: it does not flush -inf to an exact zero).
-template <int NS, int CH = 32, int EMU = 0>
-__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP,
-                                        bool poly = false) {
+template <int D>
+__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP) {
   float2 lsum2 = make_float2(0.f, 0.f);
   const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
 #pragma unroll
-  for (int part = 0; part < NS / (2 * CH); ++part) {
-    float w[CH];
+  for (int half = 0; half < 2; ++half) {
+    float w[32];
 #pragma unroll
-    for (int e = 0; e < CH; ++e) {
-      const int i = part * 2 * CH + 2 * e;
+    for (int e = 0; e < 32; ++e) {
+      const int i = half * 64 + 2 * e;
       const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
-      const float2 pv = (EMU > 0 && (e & 7) < EMU && poly)
-                            ? ex2_poly2(x)
-                            : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       lsum2 = fadd2v(lsum2, pv);
       w[e] = __uint_as_float(pack_bf16(pv.x, pv.y));
     }
-    if (CH == 32) tc::tmem_st32(tP + part * CH, w); else tc::tmem_st16(tP + part * CH, w);
+    tc::tmem_st32(tP + half * 32, w);
   }
   tc::tmem_wait_st();
   return lsum2.x + lsum2.y;
@@ -239,7 +211,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
       l_run *= alpha;
       m_run = m_new;
     }
-    const float lsum = emit_p<kBN>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS);
+    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS);
     l_run += lsum;
     tc::fence_before_sync();
     __syncwarp();
@@ -278,159 +250,16 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
   }
 }
 
-// Softmax and epilogue for one half of one head's score rows (SPLIT 2): the
-// warpgroup (hd, half) owns TMEM lanes = query rows and the score columns
-// [64 half, 64 half + 64) of its head, the P columns [32 half, 32 half + 32)
-// they turn into, and the O columns [D/2 half, D/2 half + D/2) it rescales
-// and writes.  The two halves of a row use one running maximum: per KV tile
-// each posts its part's maximum in shared memory and waits (bounded) on
-// x_full[hd] for the other's, which also orders every half's TMEM loads of S
-// before either half overwrites S with P.  Their row sums are added at the
-// end the same way.
-template <int D, bool SEG>
-__device__ __forceinline__ void softmax_half(const Params &p, Bars &bars, float *xbuf,
-                                             uint32_t tmem, int hd, int half, int b, int h,
-                                             int m0, int a0, int a_end, int lo_max, int j0,
-                                             int nt, bool *failed) {
-  using K = Cfg<D>;
-  constexpr int NC = kBN / 2;  // score columns of this half
-  constexpr int DO = D / 2;    // O columns of this half
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q4 = warp & 3;
-  const int row = q4 * 32 + lane;
-  const int t = a0 + row;       // key position of this query row
-  const int qr = m0 + row;      // its row in Q and O
-  const bool active = t < a_end;
-  const int lo_t = active ? row_lo<SEG>(p, b, t) : 0;
-  const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-  const uint32_t tS = tmem + lane_base + hd * kBN + half * NC;
-  const uint32_t tP = tmem + lane_base + hd * kBN + half * (NC / 2);
-  const uint32_t tO = tmem + lane_base + K::TM_O + hd * D + half * DO;
-  const float sc = p.scale_log2;
-  float m_run = -INFINITY, l_run = 0.f;
-  bool ok = true;
-  int xn = 0;  // exchanges so far (phase of x_full[hd])
-  // Post v, wait for the other half of the same rows, return its value.
-  auto exchange = [&](float v, float *other) -> bool {
-    float *slot = xbuf + ((xn & 1) * 4 + hd * 2) * kBM;
-    slot[half * kBM + row] = v;
-    tc::fence_before_sync();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.x_full[hd]);
-    const bool got = __all_sync(0xffffffffu, mbar_wait(&bars.x_full[hd], xn & 1, failed)) != 0;
-    tc::fence_after_sync();
-    xn++;
-    *other = slot[(1 - half) * kBM + row];
-    return got;
-  };
-  for (int j = 0; j < nt; ++j) {
-    const int kb = (j0 + j) * kBN + half * NC;  // key of this half's column 0
-    if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[hd], j & 1, failed))) { ok = false; break; }
-    tc::fence_after_sync();
-    const bool edge = (kb + NC - 1 > a0) || (kb < lo_max);
-    float s[NC];
-#pragma unroll
-    for (int c = 0; c < NC / 32; ++c) tc::tmem_ld32(tS + c * 32, s + c * 32);
-    tc::tmem_wait_ld();
-    // O and P of this head are free once its previous PV has completed.
-    if (j >= 1) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (j - 1) & 1, failed))) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-    }
-    if (edge) {
-#pragma unroll
-      for (int i = 0; i < NC; ++i) {
-        const int key = kb + i;
-        if (!(key <= t && key >= lo_t)) s[i] = -INFINITY;
-      }
-    }
-    // this half's maximum of s*scale, then the row's over both halves
-    float mx;
-    {
-      const bool neg = !(sc > 0.f);
-      float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (!neg) {
-#pragma unroll
-        for (int i = 0; i < NC; i += 2) mc[(i >> 1) & 3] = fmax3(mc[(i >> 1) & 3], s[i], s[i + 1]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < NC; ++i)
-          mc[i & 3] = fmaxf(mc[i & 3], s[i] == -INFINITY ? -INFINITY : -s[i]);
-      }
-      mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
-    }
-    float m_half = (mx == -INFINITY) ? -INFINITY : mx * fabsf(sc), m_other;
-    if (!exchange(m_half, &m_other)) { ok = false; break; }
-    const float m_tile = fmaxf(m_half, m_other);
-    if (j == 0) {
-      m_run = m_tile;
-    } else if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
-      // both halves' warps over the same rows take the same decision
-      const float m_new = fmaxf(m_run, m_tile);
-      const float alpha = m_new == m_run ? 1.f : exp2f(m_run - m_new);
-      rescale_o<DO, 16>(tO, alpha);
-      l_run *= alpha;
-      m_run = m_new;
-    }
-    constexpr int EMU = D == 64 ? GQA_PF2_EMU64 : GQA_PF2_EMU128;
-    const float lsum = emit_p<NC, 16, EMU>(s, sc, m_run == -INFINITY ? 0.f : m_run, tP, !edge);
-    l_run += lsum;
-    tc::fence_before_sync();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars.p_full[hd]);
-  }
-
-  // epilogue: O / l in bf16 over this half's columns, one row per thread
-  bool have = false;
-  if (nt > 0 && ok) {
-    have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (nt - 1) & 1, failed));
-    tc::fence_after_sync();
-  }
-  float l_other = 0.f;
-  if (have) have = exchange(l_run, &l_other);
-  const float l_row = l_run + l_other;
-  const float inv = (active && have && l_row > 0.f) ? 1.f / l_row : 0.f;
-  __nv_bfloat16 *orow = p.o + (((size_t)b * p.Hq + h) * p.Tq + min(qr, p.Tq - 1)) * D + half * DO;
-#pragma unroll
-  for (int c = 0; c < DO / 16; ++c) {
-    float ov[16];
-    if (have) {
-      tc::tmem_ld16(tO + c * 16, ov);
-      tc::tmem_wait_ld();
-    }
-    if (!have || !active) {  // inactive rows are exact zeros (their O may be NaN)
-#pragma unroll
-      for (int i = 0; i < 16; ++i) ov[i] = 0.f;
-    }
-    if (qr < p.Tq) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          w4[i] = pack_bf16(ov[e * 8 + 2 * i] * inv, ov[e * 8 + 2 * i + 1] * inv);
-        *reinterpret_cast<uint4 *>(orow + c * 16 + e * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-    }
-  }
-}
-
 // SEG: packed segment starts are given (p.seg); the plain prompt and the
 // cached-query forms compile without that code.
-template <int D, bool SEG, int SPLIT>
-__global__ void __launch_bounds__(Warps<SPLIT>::kThreads, 1)
+template <int D, bool SEG>
+__global__ void __launch_bounds__(kThreads, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const Params p) {
   using K = Cfg<D>;
-  using W = Warps<SPLIT>;
   extern __shared__ unsigned char smem_raw[];
   __shared__ Bars bars;
-  // SPLIT 2: the halves' exchanged values, [parity][head][half][row]
-  __shared__ float xbuf[SPLIT == 2 ? 2 * 2 * 2 * kBM : 1];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -445,6 +274,33 @@ __global__ void __launch_bounds__(Warps<SPLIT>::kThreads, 1)
   const int r = p.Hq / p.Hkv;
   const int h0 = g * r + 2 * pr;
   const int m0 = mt * kBM;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < K::NSLOT; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars.s_full[h], 1);
+      mbar_init(&bars.p_full[h], 4);
+      mbar_init(&bars.o_done[h], 1);
+    }
+    mbar_init(&bars.mma_fin, 1);
+    mbar_init(&bars.v_clean, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bars.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  // Barriers and TMEM are set up; from here on the CTA reads memory the
+  // previous kernel on the stream may write: wait for it (a no-op unless
+  // launched as a programmatic dependent), then let the next one start.
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   // n_b keys of sequence b; `rows` query rows produce output, the query
   // row i sits at key position off + i; a0 = position of this tile's row 0.
   int n_b = p.Tk;
@@ -481,29 +337,7 @@ __global__ void __launch_bounds__(Warps<SPLIT>::kThreads, 1)
     }
   }
 
-  if (threadIdx.x == 0) {
-    mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < K::NSLOT; ++s) {
-      mbar_init(&bars.full[s], 1);
-      mbar_init(&bars.empty[s], 1);
-    }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(&bars.s_full[h], 1);
-      mbar_init(&bars.p_full[h], 4 * SPLIT);   // every softmax warp of the head
-      mbar_init(&bars.o_done[h], 1);
-      mbar_init(&bars.x_full[h], 4 * SPLIT);
-    }
-    mbar_init(&bars.mma_fin, 1);
-    mbar_init(&bars.v_clean, 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(&bars.tmem_base, kTmemCols);
-    tc::tmem_relinquish();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
+  if (SEG) __syncthreads();  // s_lo_min / s_lo_max
   // KV tiles [j0, j0 + nt) cover the tile's permitted keys; tiles starting
   // before lo_max need masks (some row's first key lies inside them).
   int lo_min, lo_max;
@@ -530,18 +364,12 @@ __global__ void __launch_bounds__(Warps<SPLIT>::kThreads, 1)
   bool failed = false;
   if (warp >= 4) {
     // ================================================= softmax warpgroups
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(W::kRegsHigh));
-    // warps 4-7: head A, 8-11: head B (SPLIT 2: their score columns 0-63;
-    // warps 12-15 and 16-19: the same heads' columns 64-127)
-    const int hd = ((warp - 4) >> 2) & 1;
-    if (SPLIT == 1)
-      softmax_head<D, SEG>(p, bars, smem, tmem, hd, b, h0 + hd, m0, a0, off + rows, lo_max,
-                           j0, nt, &failed);
-    else
-      softmax_half<D, SEG>(p, bars, xbuf, tmem, hd, (warp - 4) >> 3, b, h0 + hd, m0, a0,
-                           off + rows, lo_max, j0, nt, &failed);
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    const int hd = (warp - 4) / 4;  // warps 4-7: head A, 8-11: head B
+    softmax_head<D, SEG>(p, bars, smem, tmem, hd, b, h0 + hd, m0, a0, off + rows, lo_max, j0,
+                         nt, &failed);
   } else {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(W::kRegsLow));
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0) {
     // ================================================= TMA producer
     if (lane == 0 && nt > 0) {
@@ -665,16 +493,6 @@ __global__ void __launch_bounds__(Warps<SPLIT>::kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host
-// Softmax warpgroups per head (1 or 2); GQA_PF2_SPLIT in the environment
-// selects one for measurements, 2 otherwise.
-inline int softmax_split() {
-  static const int v = [] {
-    const char *e = getenv("GQA_PF2_SPLIT");
-    return (e && e[0] == '1') ? 1 : 2;
-  }();
-  return v;
-}
-
 inline bool supported(int d, int Hq, int Hkv) {
   return (d == 64 || d == 128) && (Hq / Hkv) % 2 == 0;
 }
@@ -692,16 +510,10 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
     return GQA_ERR_CUDA;
   static bool attr_done = false;  // per instantiation; benign race
   if (!attr_done) {
-    if (cudaFuncSetAttribute(prefill_pair_kernel<D, false, 1>,
+    if (cudaFuncSetAttribute(prefill_pair_kernel<D, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              K::SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(prefill_pair_kernel<D, true, 1>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             K::SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(prefill_pair_kernel<D, false, 2>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             K::SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(prefill_pair_kernel<D, true, 2>,
+        cudaFuncSetAttribute(prefill_pair_kernel<D, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              K::SMEM) != cudaSuccess) {
       cudaGetLastError();
@@ -726,21 +538,16 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.scale_log2 = scale_log2;
   const long long grid = (long long)B * Hkv * p.pairs * p.num_mt;
   if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
-  const int split = softmax_split();
-  if (split == 2) {
-    constexpr int NT = Warps<2>::kThreads;
-    if (seg)
-      prefill_pair_kernel<D, true, 2><<<(unsigned)grid, NT, K::SMEM, st>>>(mq, mk, mv, p);
-    else
-      prefill_pair_kernel<D, false, 2><<<(unsigned)grid, NT, K::SMEM, st>>>(mq, mk, mv, p);
-  } else {
-    constexpr int NT = Warps<1>::kThreads;
-    if (seg)
-      prefill_pair_kernel<D, true, 1><<<(unsigned)grid, NT, K::SMEM, st>>>(mq, mk, mv, p);
-    else
-      prefill_pair_kernel<D, false, 1><<<(unsigned)grid, NT, K::SMEM, st>>>(mq, mk, mv, p);
+  const cudaError_t e =
+      seg ? launch_dependent(prefill_pair_kernel<D, true>, dim3((unsigned)grid), dim3(kThreads),
+                             K::SMEM, st, mq, mk, mv, p)
+          : launch_dependent(prefill_pair_kernel<D, false>, dim3((unsigned)grid), dim3(kThreads),
+                             K::SMEM, st, mq, mk, mv, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+  return GQA_OK;
 }
 
 // Prompt (cached = 0: Tq = Tk = T) or queries after a cache (cached = 1:

@@ -112,6 +112,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int m0 = mt * kBM;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.k_full[s], 1);
+      mbar_init(&bars.v_full[s], 1);
+      mbar_init(&bars.k_empty[s], 1);
+      mbar_init(&bars.v_empty[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.s_free[s], 4);
+    }
+    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.o_done, 1);
+    mbar_init(&bars.mma_fin, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bars.tmem_base, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  // Barriers and TMEM are set up; from here on the CTA reads memory the
+  // previous kernel on the stream may write: wait for it (a no-op unless
+  // launched as a programmatic dependent), then let the next one start.
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   // n_b keys of sequence b; `rows` query rows produce output, the query
   // row i sits at key position off + i; a0 = position of this tile's row 0.
   int n_b = p.Tk;
@@ -149,28 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (threadIdx.x == 0) {
-    mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars.k_full[s], 1);
-      mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.k_empty[s], 1);
-      mbar_init(&bars.v_empty[s], 1);
-      mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.s_free[s], 4);
-    }
-    mbar_init(&bars.p_full, 4);
-    mbar_init(&bars.o_done, 1);
-    mbar_init(&bars.mma_fin, 1);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(&bars.tmem_base, kTmemCols);
-    tc::tmem_relinquish();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
+  if (p.seg) __syncthreads();  // s_lo_min / s_lo_max
   // KV tiles [j0, j0 + nt) cover the tile's permitted keys; tiles starting
   // before lo_max need masks (some row's first key lies inside them).
   int lo_min, lo_max;
@@ -484,7 +490,11 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.scale_log2 = scale_log2;
   const long long grid = (long long)B * Hq * p.num_mt;
   if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
-  prefill_kernel<D><<<(unsigned)grid, kThreads, K::SMEM, st>>>(mq, mk, mv, p);
+  if (launch_dependent(prefill_kernel<D>, dim3((unsigned)grid), dim3(kThreads), K::SMEM, st, mq,
+                       mk, mv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return GQA_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
