@@ -7,6 +7,7 @@
 // products as in its incremental path), then kernel launches on the caller's
 // stream.  Nothing here allocates device memory.
 #include <algorithm>
+#include <cstdlib>
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -17,6 +18,7 @@
 #include "common.cuh"
 #include "decode_splitk.cuh"
 #include "prefill_pair.cuh"
+#include "prefill_split.cuh"
 #include "prefill_tc.cuh"
 #include "simt.cuh"
 
@@ -347,6 +349,13 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
   const float scale_log2 = scale * gqa::kLog2e;
   if (dtype == GQA_BF16 && gqa::pf::supported(d) && aligned16(q) &&
       aligned16(k) && aligned16(v) && aligned16(o)) {
+    static const bool split = [] {
+      const char *e = getenv("GQA_PREFILL_KERNEL");
+      return !(e && e[0] == 'p');
+    }();
+    if (split)
+      return gqa::pfs::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,
+                              window, scale_log2, dev_status, st);
     // Heads of a group in pairs (one CTA per pair) when the group size is
     // even; otherwise one head per CTA.
     if (gqa::pf2::supported(d, Hq, Hkv))
