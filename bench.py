@@ -614,9 +614,12 @@ class PrefillStep:
     def kernel(self):
         """The tensor-core kernel gqa_prefill dispatches to for this shape."""
         w = self.w
-        if w.d in (64, 128) and (w.Hq // self.Hkv) % 2 == 0:
-            return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
-        return "pf::prefill_kernel (one query head per CTA)"
+        if os.environ.get("GQA_PREFILL_KERNEL", "").startswith("p"):
+            if w.d in (64, 128) and (w.Hq // self.Hkv) % 2 == 0:
+                return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
+            return "pf::prefill_kernel (one query head per CTA)"
+        return ("pfs::prefill_split_kernel (one query head per CTA, two softmax warpgroups "
+                "of 64 score columns each)")
 
 
 def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PASSES):
@@ -634,17 +637,25 @@ def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PA
     ms = st["median_ms"] / reps
     peaks, kind = measured_peaks()
     tflops = step.flops / (ms / 1e3) / 1e12
-    return step, {
+    # The burst matmul figure is the peak for a kernel timed alone; launches
+    # back to back for a quarter of a second or more run under the power cap,
+    # which the sustained figure was measured under.
+    sustained = sum(ms_pass) > 250.0 and "bf16_tflops_sustained" in peaks
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    res = {
         **step.describe(), "kernel": step.kernel(), "tflops": round(tflops, 2), "ms": round(ms, 5),
         "launches_per_pass": reps, "passes": st["passes"],
         "pass_ms": {k: round(v, 5) for k, v in st.items() if k != "passes"},
-        "flops": step.flops, "frac_of_measured": round(tflops / peaks["bf16_tflops"], 4),
-        "peak_kind": f"{kind} bf16 matmul (burst)",
+        "timed_ms": round(sum(ms_pass), 2),
+        "flops": step.flops, "peak": peak, "frac_of_measured": round(tflops / peak, 4),
+        "peak_kind": f"{kind} bf16 matmul ({'sustained' if sustained else 'burst'})",
+        "frac_of_burst": round(tflops / peaks["bf16_tflops"], 4),
         "frac_of_spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4),
         "l2": "inputs exceed the 126 MB L2; launches back to back" if step.NL == 1 else
               f"{step.NL} copies of q, k, v and o ({step.NL * step.io_bytes / 1e6:.0f} MB in "
               f"all, above twice the 126 MB L2), launch i on copy i mod {step.NL}; launches "
               f"back to back, no flush"}
+    return step, res
 
 
 def oracle_decode_sample(step, max_seconds, single=True):
@@ -887,9 +898,10 @@ def run_gpu_prefill(args, world, rank, local):
         "data": "synthetic (seeded normal rounded to bf16)",
         "config": dict(step.describe(), parallelism=f"replicas x{world}", l2=res["l2"]),
         "roofline": {"bound": "tensor", "kernel": step.kernel(),
-                     "achieved": res["tflops"], "peak": peaks["bf16_tflops"],
-                     "peak_kind": f"{kind} bf16 matmul (burst)", "unit": "TFLOP/s",
-                     "frac": res["frac_of_measured"], "frac_of_spec_2250": res["frac_of_spec_2250"],
+                     "achieved": res["tflops"], "peak": res["peak"],
+                     "peak_kind": res["peak_kind"], "unit": "TFLOP/s",
+                     "frac": res["frac_of_measured"], "frac_of_burst": res["frac_of_burst"],
+                     "frac_of_spec_2250": res["frac_of_spec_2250"],
                      "flops_per_launch": step.flops, "avg_launch_us": round(res["ms"] * 1e3, 2),
                      "launches_per_pass": res["launches_per_pass"], "passes": res["passes"],
                      "traffic": args.traffic if args.traffic is not None else

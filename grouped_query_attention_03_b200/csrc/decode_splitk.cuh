@@ -59,24 +59,11 @@ namespace gqa {
 namespace dec {
 
 constexpr int kFirst = 1, kLast = 2, kEnd = 4;
-// Largest grid and largest number of tail chunks.  A chunk of the tail
-// counts as a virtual CTA (piece) G + k, so pieces number at most
-// kMaxCtas + kMaxTail; the workspace holds one counter per possible first
-// piece of a split lane, then the chunk counter, the count of CTAs done
-// taking chunks, and the count of CTAs that have read the lengths (fused
-// append).
+// Largest grid; the workspace holds kMaxCtas split-lane counters (a split
+// lane's first CTA indexes it) and then the count of CTAs that have read
+// the lengths (fused append).
 constexpr int kMaxCtas = 1024;
-constexpr int kMaxTail = 256;
-constexpr int kCtrGrab = kMaxCtas + kMaxTail;
-constexpr int kCtrDone = kCtrGrab + 1;
-constexpr int kCtrFinish = kCtrDone + 1;
-constexpr int kNumCounters = kCtrFinish + 1;
-// A CTA takes at most kMaxGrabs chunks (its pending split lanes then fit a
-// fixed list: two per range); the tail is used only when the split has at
-// least kTailMinStages stages per CTA.
-constexpr int kMaxGrabs = 15;
-constexpr int kMaxPend = 2 * (1 + kMaxGrabs);
-constexpr int kTailMinStages = 16;
+constexpr int kCtrFinish = kMaxCtas;
 // Lengths of up to this many sequences are cached in shared memory (read
 // from global memory once per CTA); a fused append needs that.
 constexpr int kLensSmem = 4096;
@@ -165,7 +152,6 @@ struct Params {
   int ring;       // 1: the cache is a rolling buffer of C slots, position p
                   // in slot p mod C; the query reads all min(n_b, C) slots
   int pad;        // virtual rows in front of every non-empty lane (below)
-  int tail_div;   // the tail is total / tail_div rows (0: no tail)
 };
 
 // Keys of sequence b for this call (n_b, the appended token included).
@@ -196,30 +182,6 @@ __device__ __forceinline__ int first_cell(const Params &p, int n, int len) {
 __device__ __forceinline__ int extent(const Params &p, int len) {
   return len > 0 ? len + p.pad : 0;
 }
-
-// The row split.  Rows [0, S) are split evenly: CTA c takes [c per,
-// (c + 1) per).  On large calls the last rows [S, total) are cut into nch
-// chunks of ch rows that the CTAs take one at a time from a counter in the
-// workspace as they finish (the tail: CTAs that stream faster take more of
-// it, so they finish together).  Chunk k is piece G + k: along the row
-// order the pieces (static ranges, then chunks) have increasing ids, so
-// slot = lane + id never repeats and a split lane's first piece is its own.
-struct Split {
-  long long total, S, per, ch;
-  int G, nch;
-  // first piece and number of pieces of the real rows [SR, SE)
-  __device__ __forceinline__ void pieces(long long SR, long long SE, int &c0, int &np) const {
-    int nstat = 0;
-    if (SR < S) {
-      c0 = (int)udiv(SR, per);
-      nstat = (int)udiv(min(SE, S) - 1, per) - c0 + 1;
-    } else {
-      c0 = G + (int)udiv(SR - S, ch);
-    }
-    const int ntail = SE > S ? (int)udiv(SE - 1 - S, ch) - (int)udiv(max(SR, S) - S, ch) + 1 : 0;
-    np = nstat + ntail;
-  }
-};
 
 
 // Byte offset of 16-byte chunk `ch` (0..7) of row `r` inside a 128-byte
@@ -275,27 +237,12 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
   for (int off = 16; off >= 1; off >>= 1)
     tot += __shfl_xor_sync(0xffffffffu, tot, off);
   const long long total = tot * p.VL;
-  Split sp;
-  sp.total = total;
-  sp.G = G;
-  sp.S = total;
-  sp.ch = 1;
-  sp.nch = 0;
-  if (p.tail_div > 0 && total >= (long long)G * kTailMinStages * K::ROWS) {
-    const long long tail = udiv(total, p.tail_div);
-    const long long maxch = min((long long)kMaxTail, (long long)G * kMaxGrabs);
-    long long ch = 2 * K::ROWS;
-    if (tail > ch * maxch) ch = udiv(udiv(tail + maxch - 1, maxch) + K::ROWS - 1, K::ROWS) * K::ROWS;
-    sp.ch = ch;
-    sp.nch = (int)udiv(tail + ch - 1, ch);
-    sp.S = total - tail;
-  }
-  long long per = udiv(sp.S + G - 1, G);
+  long long per = udiv(total + G - 1, G);
   if (per < p.min_rows) per = p.min_rows;
-  sp.per = per;
+  const long long start = (long long)c * per;
+  const long long end = min(total, start + per);
 
-  // Walk rows [start, end) as piece `vid`; false if a ring wait gave up.
-  auto walk = [&](long long start, long long end, int vid) -> bool {
+  if (!bad && start < end) {
     // Pass 2: find the batch row holding row `start` (warp prefix scan).
     long long cum = 0, cum_b = 0;
     int b = -1;
@@ -318,7 +265,6 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
         cum += __shfl_sync(0xffffffffu, incl, 31);
       }
     }
-    if (b < 0) return true;  // start lies past every row (not reached)
     int n_b = len_of(b);
     int len = eligible_cells(p, n_b);
     int ext = extent(p, len);
@@ -340,15 +286,16 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
       const int nrows = (int)min((long long)min(K::ROWS, len - row), end - pos);
       const bool last = (row + nrows == len) || (pos + nrows == end);
       int st;
-      if (!acquire(st)) return false;
+      if (!acquire(st)) break;
       if (lane == 0) {
         StageHdr &h = hdrs[st];
         h.lane = L;
         h.cell0 = lo + row;
         h.nrows = nrows;
         h.flags = (seg_first ? kFirst : 0) | (last ? kLast : 0);
-        h.slot = L + vid;
-        sp.pieces(SR, SR + len, h.c0, h.np);
+        h.slot = L + c;
+        h.c0 = (int)udiv(SR, per);
+        h.np = (int)udiv(SR + len - 1, per) - h.c0 + 1;
         // the appended token's cell: the last one, or (ring) its slot
         const int cnew = p.ring ? (n_b - 1) % p.C : n_b - 1;
         h.newrow = (p.add && cnew >= lo + row && cnew < lo + row + nrows) ? cnew - lo - row : -1;
@@ -408,29 +355,6 @@ __device__ void producer(const Params &p, const CUtensorMap *tmK,
           lo = first_cell(p, n_b, len);
         }
       }
-    }
-    return true;
-  };
-
-  if (!bad) {
-    const long long s0 = (long long)c * per, e0 = min(sp.S, s0 + per);
-    bool ok = s0 < e0 ? walk(s0, e0, c) : true;
-    if (sp.nch > 0) {
-      // the tail: take chunks until none is left (or this CTA's share is
-      // used up), then count this CTA done; the last one resets both counts
-      for (int grabs = 0; ok && grabs < kMaxGrabs; ++grabs) {
-        int k = 0;
-        if (lane == 0) k = atomicAdd(&p.counters[kCtrGrab], 1);
-        k = __shfl_sync(0xffffffffu, k, 0);
-        if (k >= sp.nch) break;
-        const long long a = sp.S + (long long)k * sp.ch;
-        ok = walk(a, min(sp.total, a + sp.ch), G + k);
-      }
-      if (lane == 0 && atomicAdd(&p.counters[kCtrDone], 1) == G - 1) {
-        p.counters[kCtrGrab] = 0;
-        p.counters[kCtrDone] = 0;
-      }
-      __syncwarp();
     }
   }
   // End marker.
@@ -576,15 +500,10 @@ __device__ __noinline__ void merge_lane(const Params &p, int L, int c0, int np,
 //   B regs 0..1: (rows 2t..2t+1, col g), (rows 8+2t.., col g)
 //   C regs 0..3: (row g, cols 2t, 2t+1), (row g+8, cols 2t, 2t+1)
 // Tile rows are query heads; S columns are cache rows; O columns features.
-// A split lane whose partial this CTA wrote: counted at the end of the CTA.
-struct Pend {
-  int lane, c0, np;
-};
-
 template <int D, int R>
 __device__ void consumer(const Params &p, unsigned char *smem,
                          const StageHdr *hdrs, uint64_t *full, uint64_t *empty,
-                         uint64_t *comb, Pend *pend, int *merge_cnt) {
+                         uint64_t *comb, int &merge_flag) {
   using K = Cfg<D, R>;
   constexpr int NWC = K::NWC, KS = K::KS, NT = K::NT;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -595,10 +514,9 @@ __device__ void consumer(const Params &p, unsigned char *smem,
   float o[NT][4];          // O tile accumulators
   float m_run[2], l_run[2];  // head rows g and g + 8
   int stage_count = 0, comb_count = 0;
-  // Split lanes whose partial this CTA wrote are listed in `pend` (by
-  // thread 0; every compute thread sees the same stage headers) and counted
-  // at the end: at most two per range (its first and last segment).
-  int pend_n = 0;
+  // Split lanes whose partial this CTA wrote, counted at the end (at most
+  // two: the first and the last segment of the range).
+  int pend_n = 0, pL0 = 0, pc0 = 0, pn0 = 0, pL1 = 0, pc1 = 0, pn1 = 0;
 
   while (true) {
     const int st = stage_count % K::STAGES;
@@ -813,11 +731,16 @@ __device__ void consumer(const Params &p, unsigned char *smem,
             tc::st_global_hint(&p.ml[(size_t)hd.slot * R + h], make_float2(mm, lsum), keep);
         }
       }
-      // A partial is counted at the end of the CTA's work: nobody needs it
+      // A partial is counted at the end of the CTA's range: nobody needs it
       // sooner (the lane's other pieces end with their CTAs' ranges), and the
-      // warps go on to the next segment without waiting for the count.
-      if (hd.np > 1 && pend_n < kMaxPend) {
-        if (threadIdx.x == 0) pend[pend_n] = Pend{L, hd.c0, hd.np};
+      // warps go on to the next segment without waiting for the count.  A
+      // range has at most two split lanes, its first and its last.
+      if (hd.np > 1 && pend_n < 2) {
+        if (pend_n == 0) {
+          pL0 = L; pc0 = hd.c0; pn0 = hd.np;
+        } else {
+          pL1 = L; pc1 = hd.c0; pn1 = hd.np;
+        }
         pend_n++;
       }
     }
@@ -831,48 +754,37 @@ __device__ void consumer(const Params &p, unsigned char *smem,
     // last to finish.  After the barrier one thread's release fence covers
     // the stores of the whole CTA; its acquire fence (when last) covers the
     // loads of the merges, which every thread starts after the second
-    // barrier.  The lanes to merge go to the front of the list.
+    // barrier.
     csync(comb, comb_count, &failed);
     if (threadIdx.x == 0) {
       fence_acq_rel_gpu();
-      int nm = 0;
-      for (int i = 0; i < pend_n; ++i) {
-        const Pend e = pend[i];
-        if (atomicAdd(&p.counters[e.c0], 1) == e.np - 1) {
-          // the lane's last count is its counter's last access in this
-          // call: leave it zero for the next call
-          p.counters[e.c0] = 0;
-          pend[nm++] = e;
-        }
-      }
-      if (nm) fence_acq_rel_gpu();
-      *merge_cnt = nm;
+      const int o0 = atomicAdd(&p.counters[pc0], 1);
+      const int o1 = pend_n > 1 ? atomicAdd(&p.counters[pc1], 1) : 0;
+      const int flags = (o0 == pn0 - 1 ? 1 : 0) | (pend_n > 1 && o1 == pn1 - 1 ? 2 : 0);
+      // The last count of a lane is its counter's last access in this call:
+      // leave it zero for the next call.
+      if (flags & 1) p.counters[pc0] = 0;
+      if (flags & 2) p.counters[pc1] = 0;
+      if (flags) fence_acq_rel_gpu();
+      merge_flag = flags;
     }
     csync(comb, comb_count, &failed);
-    const int nm = *merge_cnt;
-    auto out_of = [&](int L, int &rc) {
-      const int b = L / p.VL, vl = L % p.VL;
+    const int flags = merge_flag;
+    // Two merges run side by side (warps 0-3 and the rest), one runs on
+    // every compute warp.
+    constexpr int NA = 4 * 32, NBT = (NWC - 4) * 32;
+    const int i = flags == 3 ? (w < 4 ? 0 : 1) : (flags == 2 ? 1 : 0);
+    if (flags) {
+      const int L = i ? pL1 : pL0, b = L / p.VL, vl = L % p.VL;
       const int h0 = (vl / p.nsub) * p.r + (vl % p.nsub) * R;
-      rc = min(R, p.r - (vl % p.nsub) * R);
-      return p.o + ((size_t)b * p.Hq + h0) * D;
-    };
-    if (nm == 2) {
-      // two merges side by side (warps 0-3 and the rest)
-      constexpr int NA = 4 * 32, NBT = (NWC - 4) * 32;
-      const Pend e = pend[w < 4 ? 0 : 1];
-      int rc;
-      __nv_bfloat16 *out = out_of(e.lane, rc);
-      if (w < 4)
-        merge_lane<D, R, NA>(p, e.lane, e.c0, e.np, out, rc, threadIdx.x);
+      const int rc = min(R, p.r - (vl % p.nsub) * R);
+      __nv_bfloat16 *out = p.o + ((size_t)b * p.Hq + h0) * D;
+      if (flags != 3)
+        merge_lane<D, R, NWC * 32>(p, L, i ? pc1 : pc0, i ? pn1 : pn0, out, rc, threadIdx.x);
+      else if (w < 4)
+        merge_lane<D, R, NA>(p, L, pc0, pn0, out, rc, threadIdx.x);
       else
-        merge_lane<D, R, NBT>(p, e.lane, e.c0, e.np, out, rc, threadIdx.x - NA);
-    } else {
-      for (int i = 0; i < nm; ++i) {
-        const Pend e = pend[i];
-        int rc;
-        __nv_bfloat16 *out = out_of(e.lane, rc);
-        merge_lane<D, R, NWC * 32>(p, e.lane, e.c0, e.np, out, rc, threadIdx.x);
-      }
+        merge_lane<D, R, NBT>(p, L, pc1, pn1, out, rc, threadIdx.x - NA);
     }
   }
   if (failed && lane == 0) record_status(p.status, kStatusTimeout);
@@ -881,13 +793,17 @@ __device__ void consumer(const Params &p, unsigned char *smem,
 template <int D, int R>
 __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
     split_kernel(const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const Params p) {
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params pk) {
   using K = Cfg<D, R>;
   extern __shared__ unsigned char smem_raw[];
+  // The parameters, copied to shared memory by one warp's parallel loads at
+  // entry: read from the parameter bank instead, each first touch of one of
+  // its cache lines stalls the (single) producer warp on the way to its
+  // first copy.
+  __shared__ __align__(16) Params sp;
   __shared__ StageHdr hdrs[K::STAGES];
   __shared__ __align__(8) uint64_t full[K::STAGES], empty[K::STAGES], comb;
-  __shared__ int merge_cnt, s_bad;
-  __shared__ Pend pend[kMaxPend];
+  __shared__ int merge_flag, s_bad;
   __shared__ __align__(8) uint64_t lens_ready;
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -907,7 +823,13 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
     tc::prefetch_tmap(&tmK);
     tc::prefetch_tmap(&tmV);
   }
+  if (warp == 0) {
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(&pk);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(&sp);
+    for (int i = lane; i < (int)(sizeof(Params) / 4); i += 32) dst[i] = src[i];
+  }
   __syncthreads();
+  const Params &p = sp;
   // Everything above touches only shared memory and the kernel parameters.
   // From here on the CTA reads and writes global memory that the previous
   // kernel on the stream may use: wait until it has completed (a no-op when
@@ -952,7 +874,7 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
       for (int i = threadIdx.x; i < p.Hq * D / 8; i += K::NWC * 32)
         reinterpret_cast<uint4 *>(ob)[i] = make_uint4(0, 0, 0, 0);
     }
-    consumer<D, R>(p, smem, hdrs, full, empty, &comb, pend, &merge_cnt);
+    consumer<D, R>(p, smem, hdrs, full, empty, &comb, merge_flag);
   }
 }
 

@@ -37,12 +37,7 @@ constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;  // smallest row range per CTA
 // A lane segment's fixed cost in a CTA, as cache bytes: the split gives each
 // non-empty lane this many bytes of virtual rows (see dec::extent).
 constexpr int kDecodeLanePadBytes = GQA_DEC_LANE_PAD_BYTES;
-#ifndef GQA_DEC_TAIL_DIV
-#define GQA_DEC_TAIL_DIV 16
-#endif
-// On large calls the last 1/kDecodeTailDiv of the rows is handed out in
-// chunks to the CTAs that finish first (0: no tail).
-constexpr int kDecodeTailDiv = GQA_DEC_TAIL_DIV;
+
 
 struct DeviceInfo {
   int sms = 0;
@@ -138,20 +133,20 @@ struct DecLayout {
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace: the counters (one per possible first piece of a split lane,
-// the tail's chunk counter and done count, and the count of CTAs that have
-// read the lengths) at a fixed place for every shape, zero between calls;
-// then the (m, l) and acc partials, one slot per (lane, piece) pair.
+// Workspace: the arrival counters (one per possible first CTA of a split
+// lane, and one count of CTAs that have read the lengths) at a fixed place
+// for every shape, zero between calls; then the (m, l) and acc partials, one
+// slot per (lane, CTA) pair touching it.
 bool decode_layout(int B, int Hq, int Hkv, int d, DecLayout *L) {
   const DecPlan pl = decode_plan(Hq, Hkv);
   int64_t lanes, slots, ml_elems, acc_elems;
   if (!elems(&lanes, {B, pl.VL})) return false;
-  slots = lanes + kMaxDecodeCtas + gqa::dec::kMaxTail;
+  slots = lanes + kMaxDecodeCtas;
   if (!elems(&ml_elems, {slots, pl.R})) return false;
   if (!elems(&acc_elems, {slots, pl.R, d})) return false;
   if (acc_elems > INT64_MAX / 8) return false;
   L->counters = 0;
-  L->counter_bytes = (size_t)gqa::dec::kNumCounters * sizeof(int);
+  L->counter_bytes = (size_t)(gqa::dec::kCtrFinish + 1) * sizeof(int);
   L->ml = round256(L->counter_bytes);
   L->acc = L->ml + round256((size_t)ml_elems * sizeof(float2));
   L->total = L->acc + round256((size_t)acc_elems * sizeof(float));
@@ -500,7 +495,6 @@ gqa_status decode_impl(gqa_dtype dtype, const void *q, const void *k_cache,
     p.lens_smem = B <= gqa::dec::kLensSmem ? 1 : 0;
     p.ring = (ap && ap->ring) ? 1 : 0;
     p.pad = kDecodeLanePadBytes / (4 * d);  // K and V rows of d bf16
-    p.tail_div = kDecodeTailDiv;
     if (clear_counters &&
         cudaMemsetAsync(p.counters, 0, L.counter_bytes, st) != cudaSuccess) {
       cudaGetLastError();

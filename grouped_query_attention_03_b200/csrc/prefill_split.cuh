@@ -112,21 +112,33 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_split_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
-                         const __grid_constant__ CUtensorMap tmV, const Params p) {
+                         const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ Params pk) {
   using K = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
+  // The parameters, copied to shared memory by one warp's parallel loads at
+  // entry (each first touch of a parameter-bank cache line would otherwise
+  // stall the warp that makes it).
+  __shared__ __align__(16) Params sp;
   __shared__ Bars bars;
   __shared__ float xbuf[2 * 2 * kBM];  // [exchange parity][half][row]
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  if (warp == 2) {
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(&pk);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(&sp);
+    for (int i = lane; i < (int)(sizeof(Params) / 4); i += 32) dst[i] = src[i];
+  }
+  const Params &p = sp;
+
   // ---- which tile: longest causal rows first; heads of a KV group adjacent
-  const int BH = p.B * p.Hq;
-  const int mt = p.num_mt - 1 - (int)(blockIdx.x / BH);
+  const int BH = pk.B * pk.Hq;
+  const int mt = pk.num_mt - 1 - (int)(blockIdx.x / BH);
   const int bh = (int)(blockIdx.x % BH);
-  const int b = bh / p.Hq, h = bh - b * p.Hq;
-  const int g = h / (p.Hq / p.Hkv);
+  const int b = bh / pk.Hq, h = bh - b * pk.Hq;
+  const int g = h / (pk.Hq / pk.Hkv);
   const int m0 = mt * kBM;
 
   if (threadIdx.x == 0) {

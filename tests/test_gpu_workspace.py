@@ -25,7 +25,7 @@ from grouped_query_attention_03_b200 import synthetic
 pytestmark = pytest.mark.gpu
 
 DEV = torch.device("cuda:0")
-COUNTER_BYTES = (1024 + 256 + 3) * 4   # first-piece counters, chunk and done counts, lengths-read count
+COUNTER_BYTES = (1024 + 1) * 4   # split-lane counters + the lengths-read count
 
 SHAPES = [
     # (B, Hq, Hkv, C, d, lengths, window)
