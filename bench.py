@@ -614,10 +614,8 @@ class PrefillStep:
     def kernel(self):
         """The tensor-core kernel gqa_prefill dispatches to for this shape."""
         w = self.w
-        if os.environ.get("GQA_PREFILL_KERNEL", "").startswith("p"):
-            if w.d in (64, 128) and (w.Hq // self.Hkv) % 2 == 0:
-                return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
-            return "pf::prefill_kernel (one query head per CTA)"
+        if w.d in (64, 128) and (w.Hq // self.Hkv) % 2 == 0:
+            return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
         return ("pfs::prefill_split_kernel (one query head per CTA, two softmax warpgroups "
                 "of 64 score columns each)")
 

@@ -793,14 +793,9 @@ __device__ void consumer(const Params &p, unsigned char *smem,
 template <int D, int R>
 __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
     split_kernel(const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params pk) {
+                 const __grid_constant__ CUtensorMap tmV, const Params p) {
   using K = Cfg<D, R>;
   extern __shared__ unsigned char smem_raw[];
-  // The parameters, copied to shared memory by one warp's parallel loads at
-  // entry: read from the parameter bank instead, each first touch of one of
-  // its cache lines stalls the (single) producer warp on the way to its
-  // first copy.
-  __shared__ __align__(16) Params sp;
   __shared__ StageHdr hdrs[K::STAGES];
   __shared__ __align__(8) uint64_t full[K::STAGES], empty[K::STAGES], comb;
   __shared__ int merge_flag, s_bad;
@@ -823,13 +818,7 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
     tc::prefetch_tmap(&tmK);
     tc::prefetch_tmap(&tmV);
   }
-  if (warp == 0) {
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(&pk);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(&sp);
-    for (int i = lane; i < (int)(sizeof(Params) / 4); i += 32) dst[i] = src[i];
-  }
   __syncthreads();
-  const Params &p = sp;
   // Everything above touches only shared memory and the kernel parameters.
   // From here on the CTA reads and writes global memory that the previous
   // kernel on the stream may use: wait until it has completed (a no-op when

@@ -7,7 +7,6 @@
 // products as in its incremental path), then kernel launches on the caller's
 // stream.  Nothing here allocates device memory.
 #include <algorithm>
-#include <cstdlib>
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -19,7 +18,6 @@
 #include "decode_splitk.cuh"
 #include "prefill_pair.cuh"
 #include "prefill_split.cuh"
-#include "prefill_tc.cuh"
 #include "simt.cuh"
 
 namespace {
@@ -342,22 +340,16 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
   if ((s = device_info(&di)) != GQA_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const float scale_log2 = scale * gqa::kLog2e;
-  if (dtype == GQA_BF16 && gqa::pf::supported(d) && aligned16(q) &&
+  if (dtype == GQA_BF16 && gqa::pfs::supported(d) && aligned16(q) &&
       aligned16(k) && aligned16(v) && aligned16(o)) {
-    static const bool split = [] {
-      const char *e = getenv("GQA_PREFILL_KERNEL");
-      return !(e && e[0] == 'p');
-    }();
-    if (split)
-      return gqa::pfs::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,
-                              window, scale_log2, dev_status, st);
-    // Heads of a group in pairs (one CTA per pair) when the group size is
-    // even; otherwise one head per CTA.
+    // Heads of a group in pairs (one CTA per pair, each K/V tile fetched
+    // once for both) when the group size is even; otherwise one head per
+    // CTA, its score rows split over two softmax warpgroups.
     if (gqa::pf2::supported(d, Hq, Hkv))
       return gqa::pf2::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached,
                               d, window, scale_log2, dev_status, st);
-    return gqa::pf::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,
-                           window, scale_log2, dev_status, st);
+    return gqa::pfs::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,
+                            window, scale_log2, dev_status, st);
   }
   if (Hq > 65535 || B > 65535) return GQA_ERR_UNSUPPORTED;
   if (dtype == GQA_F32)

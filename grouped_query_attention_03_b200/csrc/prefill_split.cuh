@@ -2,13 +2,14 @@
 // head per CTA, each score row shared by two softmax warpgroups (bf16,
 // sm_100a).
 //
-// What it computes is what prefill_tc.cuh computes ("Share key/value heads
-// and make context explicit", sections "Give each query head an explicit
-// shared KV head" and "Intersect the window with the context already
-// permitted"; FlashAttention's running max/sum from "GQA, FlashAttention and
-// the KV cache"): for every batch row b, query head h and active cell
-// t < n_b, softmax over the permitted keys of scale * q.k, mixed with the
-// value rows of the shared lane g(h); inactive rows are zero.
+// What it computes ("Share key/value heads and make context explicit",
+// sections "Give each query head an explicit shared KV head" and "Intersect
+// the window with the context already permitted"; FlashAttention's running
+// max/sum from "GQA, FlashAttention and the KV cache"): for every batch row
+// b, query head h and active cell t < n_b, softmax over the permitted keys
+// of scale * q.k, mixed with the value rows of the shared lane g(h);
+// inactive rows are zero.  It serves group sizes the paired kernel
+// (prefill_pair.cuh) cannot: odd ones, MHA included.
 //
 // One CTA owns a 128-row query tile of one (b, h) and walks the 128-key
 // tiles that intersect its permitted band, skipping tiles wholly outside
@@ -112,33 +113,21 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_split_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
-                         const __grid_constant__ CUtensorMap tmV,
-                         const __grid_constant__ Params pk) {
+                         const __grid_constant__ CUtensorMap tmV, const Params p) {
   using K = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
-  // The parameters, copied to shared memory by one warp's parallel loads at
-  // entry (each first touch of a parameter-bank cache line would otherwise
-  // stall the warp that makes it).
-  __shared__ __align__(16) Params sp;
   __shared__ Bars bars;
   __shared__ float xbuf[2 * 2 * kBM];  // [exchange parity][half][row]
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (warp == 2) {
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(&pk);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(&sp);
-    for (int i = lane; i < (int)(sizeof(Params) / 4); i += 32) dst[i] = src[i];
-  }
-  const Params &p = sp;
-
   // ---- which tile: longest causal rows first; heads of a KV group adjacent
-  const int BH = pk.B * pk.Hq;
-  const int mt = pk.num_mt - 1 - (int)(blockIdx.x / BH);
+  const int BH = p.B * p.Hq;
+  const int mt = p.num_mt - 1 - (int)(blockIdx.x / BH);
   const int bh = (int)(blockIdx.x % BH);
-  const int b = bh / pk.Hq, h = bh - b * pk.Hq;
-  const int g = h / (pk.Hq / pk.Hkv);
+  const int b = bh / p.Hq, h = bh - b * p.Hq;
+  const int g = h / (p.Hq / p.Hkv);
   const int m0 = mt * kBM;
 
   if (threadIdx.x == 0) {
