@@ -631,6 +631,22 @@ def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PA
     graph = capture(lambda: [step.run(i) for i in range(reps)], device)
     ms_pass = repeat_passes(lambda: timed(graph.replay, device), device, min_passes)
     del graph
+    alone = None
+    if step.NL == 1:
+        # The same launch timed alone, the GPU idle for a few ms before each
+        # (clocks as for a single call, the burst matmul figure's condition).
+        g1 = capture(lambda: step.run(0), device)
+        one = []
+        for _ in range(max(5, min(reps, 20))):
+            time.sleep(0.003)
+            one.append(timed(g1.replay, device))
+        del g1
+        one = dist_max_list(one, device)
+        ms1 = statistics.median(one)
+        tf1 = step.flops / (ms1 / 1e3) / 1e12
+        alone = {"tflops": round(tf1, 2), "us": round(ms1 * 1e3, 2), "launches": len(one),
+                 "frac_of_burst": round(tf1 / measured_peaks()[0]["bf16_tflops"], 4),
+                 "what": "single launches, the GPU idle 3 ms before each; median"}
     st = pass_stats(ms_pass)
     ms = st["median_ms"] / reps
     peaks, kind = measured_peaks()
@@ -649,6 +665,7 @@ def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PA
         "peak_kind": f"{kind} bf16 matmul ({'sustained' if sustained else 'burst'})",
         "frac_of_burst": round(tflops / peaks["bf16_tflops"], 4),
         "frac_of_spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4),
+        "alone": alone,
         "l2": "inputs exceed the 126 MB L2; launches back to back" if step.NL == 1 else
               f"{step.NL} copies of q, k, v and o ({step.NL * step.io_bytes / 1e6:.0f} MB in "
               f"all, above twice the 126 MB L2), launch i on copy i mod {step.NL}; launches "

@@ -273,29 +273,4 @@ __device__ __forceinline__ float2 fadd2v(float2 a, float2 b) {
       : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
   return *reinterpret_cast<float2 *>(&d);
 }
-
-// 2^x for a pair of values on the FMA and integer pipes instead of the
-// special-function unit.  Method (Cody and Waite's argument reduction): x =
-// j + f with j = round(x), found by adding and subtracting 1.5 * 2^23, and
-// f in [-1/2, 1/2]; 2^f from a cubic whose coefficients were fitted to
-// minimise the relative error on that interval by iteratively reweighted
-// least squares (largest relative error 7.5e-5 in fp32, against 2^-9 for
-// the bf16 rounding that follows); 2^j added to the exponent field.  Inputs
-// are clamped to x >= -126, so there is no flush to zero: callers keep
-// masked (-inf) cells on ex2_approx.
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  constexpr float kC0 = 0.99992805719f, kC1 = 0.69326096773f;
-  constexpr float kC2 = 0.24261114001f, kC3 = 0.05517165735f;
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
-  const float2 t = fadd2v(x, make_float2(kRound, kRound));  // kRound + j
-  const float2 j = fadd2v(t, make_float2(-kRound, -kRound));
-  const float2 f = ffma2v(j, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2v(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = ffma2v(p, f, make_float2(kC1, kC1));
-  p = ffma2v(p, f, make_float2(kC0, kC0));
-  // the low bits of t hold j (two's complement), so t << 23 is j << 23
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
 }  // namespace gqa

@@ -26,9 +26,12 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kMaxDecodeCtas = gqa::dec::kMaxCtas;  // workspace is sized for this many
 #ifndef GQA_DEC_MIN_ROWS
-#define GQA_DEC_MIN_ROWS 256
+#define GQA_DEC_MIN_ROWS 320
 #endif
-constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;  // smallest row range per CTA
+// Smallest row range per CTA: small calls use fewer CTAs, so that a lane is
+// split into at most about 16 partials, which the merge reads in one batch
+// (swept 256-384 on the 16.8 MB sliding-window step: 320 fastest).
+constexpr int kDecodeMinRows = GQA_DEC_MIN_ROWS;
 #ifndef GQA_DEC_LANE_PAD_BYTES
 #define GQA_DEC_LANE_PAD_BYTES 131072
 #endif

@@ -48,11 +48,6 @@ constexpr int kThreads = 384;
 // issuer, two idle warps) gives registers to the two softmax warpgroups.
 // 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * (launch registers).
 constexpr int kRegsLow = 72, kRegsHigh = 216;
-// Pairs of every 8 whose exponentials the softmax computes on the FMA pipe
-// (tiles with no masked cell only).
-#ifndef GQA_PF2_EMU
-#define GQA_PF2_EMU 0
-#endif
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 12;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -127,11 +122,8 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 // unit; masked cells give exactly 0), written as bf16 P into this thread's
 // TMEM lane over the S columns it came from (column c holds p[2c], p[2c+1]),
 // where the P V MMA reads it as its A operand; returns the row sum.
-// With `poly` (a tile whose cells are all permitted), EMU of every 8 pairs
-// take the FMA-pipe exponential, relieving the special-function unit.
-template <int D, int EMU = 0>
-__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP,
-                                        bool poly = false) {
+template <int D>
+__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP) {
   float2 lsum2 = make_float2(0.f, 0.f);
   const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
 #pragma unroll
@@ -141,9 +133,7 @@ __device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint3
     for (int e = 0; e < 32; ++e) {
       const int i = half * 64 + 2 * e;
       const float2 x = ffma2v(make_float2(s[i], s[i + 1]), sc2, nm2);
-      const float2 pv = (EMU > 0 && (e & 7) < EMU && poly)
-                            ? ex2_poly2(x)
-                            : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
       lsum2 = fadd2v(lsum2, pv);
       w[e] = __uint_as_float(pack_bf16(pv.x, pv.y));
     }
@@ -224,7 +214,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
       l_run *= alpha;
       m_run = m_new;
     }
-    const float lsum = emit_p<D, GQA_PF2_EMU>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS, !edge);
+    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS);
     l_run += lsum;
     tc::fence_before_sync();
     __syncwarp();
