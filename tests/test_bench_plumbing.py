@@ -91,3 +91,33 @@ def test_pass_count_covers_minimum_passes_and_time():
     assert bench.n_passes(100.0, cpu, min_passes=30, min_seconds=0.5) == 30
     # never more than the cap
     assert bench.n_passes(1e-6, cpu, min_passes=30, min_seconds=10.0) == 3000
+
+
+def test_copy_count_keeps_steps_out_of_l2():
+    """Inputs above the 126 MB L2 need no copies; smaller ones get enough
+    copies that the copies together hold more than twice the L2."""
+    assert bench.n_copies(262_000_000) == 1
+    assert bench.n_copies(127_000_000) == 1
+    for b in (16_777_216, 10_485_760, 1_000_000):
+        n = bench.n_copies(b)
+        assert n * b > 2 * bench.L2_BYTES or n == 64
+        assert (n - 2) * b <= 2 * bench.L2_BYTES  # not more than one copy beyond that
+
+
+def test_loop_bytes_count_each_copy_growth():
+    """Call i of the successive-calls loop runs on copy i mod NL, which has
+    grown by i // NL cells; with a window the bytes stop growing."""
+    import numpy as np
+    from grouped_query_attention_03_b200 import workloads
+    s = bench.DecodeStep.__new__(bench.DecodeStep)
+    s.w, s.Hkv, s.window, s.cached = workloads.DECODE_B8_N8000, 8, None, [8000] * 8
+    s.qo_bytes, s.write_bytes, s.NL = 1000, 100, 1
+    per_cell = 2 * 8 * 8 * 128 * 2       # K+V bytes of one more cell in every sequence
+    base = s.step_bytes_at(0)
+    assert s.loop_bytes(3) == 3 * base + (0 + 1 + 2) * per_cell
+    s.NL = 2                             # calls 0,1 at +0 cells, 2,3 at +1, 4 at +2
+    assert s.loop_bytes(5) == 5 * base + (0 + 0 + 1 + 1 + 2) * per_cell
+    s.window, s.cached = 4096, [32768]   # window-capped: every call reads 4096 cells
+    s.w = workloads.SWA_T32768
+    assert s.kv_bytes_at(0) == s.kv_bytes_at(63) == 2 * 8 * 4096 * 128 * 2
+    assert np.isclose(s.loop_bytes(64), 64 * s.step_bytes_at(0))

@@ -301,13 +301,17 @@ def test_swa_t32768_decode_steps(cuda_lib):
     assert int(st.item()) == 0 and lens.tolist() == [C]
 
 
-def test_prefill_swa_t32768_sampled_rows(cuda_lib):
-    """Sliding-window prefill at full size (B=1, Hq=32, Hkv=8, d=128,
-    T=32768, w=4096), checked on a stratified sample the oracle computes row
+@pytest.mark.parametrize("Hkv", [8, 32], ids=["gqa", "mha"])
+def test_prefill_swa_t32768_sampled_rows(cuda_lib, Hkv):
+    """Sliding-window prefill at full size (B=1, Hq=32, d=128, T=32768,
+    w=4096; Hkv=8 runs the paired kernel, the MHA endpoint Hkv=32 the
+    split-row kernel), checked on a stratified sample the oracle computes row
     by row: every row t < 4096 of heads 0 and 31 (the window's ramp), and all
     32 heads at 64 seeded random cells."""
     w = workloads.SWA_T32768
     window = w.windows[0]
+    w = workloads.Workload(w.name, w.dtype, B=w.B, Hq=w.Hq, Hkv=Hkv, d=w.d, T=w.T,
+                           windows=w.windows, std=w.std, seed=w.seed)
     q, k, v = synthetic.qkv_prefill(w.B, w.Hq, w.Hkv, w.T, w.d, w.seed, std=w.std)
     o = cuda_lib.prefill(*_cuda(q, k, v), window=window)
     torch.cuda.synchronize()
