@@ -161,21 +161,29 @@ def pass_stats(ms):
 
 
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu
-# captures (the committed summaries name the workload and the kernel), keyed
-# by (workload, phase).  Each holds the SHA-256 of the kernel's source files
-# at capture time, comments and blank lines stripped: once the code changes
-# the figure no longer describes the kernel and is reported as null (a
-# comment edit does not count).
-CAPTURED_TRAFFIC = {
-    ("decode_b8_n8000", "decode"): {
-        "bytes": 268_888_576, "window": None, "hkv": None,
-        "sources": ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "469e7abd4723ef10c25be45c3b3cbd9aa34bb86e61b8ae0969f0048e75fed2f6"},
-    ("swa_t32768", "prefill"): {
-        "bytes": 692_894_976, "window": 4096, "hkv": None,
-        "sources": ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"],
-        "sha256": "8c21ff11fc3aa0eda24d66f6c45b5c1a8fec2dec9750684743198082896bf26a"},
-}
+# captures (the committed summaries name the workload and the kernel), per
+# (workload, phase, window, Hkv) as the bench is invoked.  Each holds the
+# SHA-256 of the kernel's source files at capture time, comments and blank
+# lines stripped: once the code changes the figure no longer describes the
+# kernel and is reported as null (a comment edit does not count).
+DECODE_SOURCES = ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"]
+DECODE_SHA = "b36d81a54f38f0e6833eb54afe7b30de32d3c5f26ca7ac64b09690ae6d3fce86"
+PAIR_SOURCES = ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"]
+PAIR_SHA = "9740e0e8f139f060b772d940e3574914bc539b1d9dd876077a68a9a064320963"
+CAPTURED_TRAFFIC = [
+    {"workload": "decode_b8_n8000", "phase": "decode", "window": None, "hkv": None,
+     "bytes": 267_997_440, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+    {"workload": "decode_ragged", "phase": "decode", "window": None, "hkv": 1,
+     "bytes": 148_572_928, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+    {"workload": "decode_ragged", "phase": "decode", "window": None, "hkv": 8,
+     "bytes": 1_124_909_120, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+    {"workload": "swa_t32768", "phase": "decode", "window": None, "hkv": None,
+     "bytes": 17_122_304, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+    {"workload": "prefill_b4_t1024", "phase": "prefill", "window": None, "hkv": None,
+     "bytes": 6_350_848, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+    {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": None,
+     "bytes": 691_728_640, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+]
 
 
 def strip_comments(src):
@@ -215,8 +223,9 @@ def source_digest(texts):
 def captured_traffic(workload, phase, window, hkv):
     """ncu DRAM bytes per launch for this workload if the kernel's code (its
     sources without comments) is the captured code, else None."""
-    c = CAPTURED_TRAFFIC.get((workload, phase))
-    if c is None or window != c["window"] or hkv != c["hkv"]:
+    c = next((e for e in CAPTURED_TRAFFIC if (e["workload"], e["phase"], e["window"], e["hkv"])
+              == (workload, phase, window, hkv)), None)
+    if c is None:
         return None
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)),
                         "grouped_query_attention_03_b200", "csrc")
@@ -666,6 +675,7 @@ def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PA
         "frac_of_burst": round(tflops / peaks["bf16_tflops"], 4),
         "frac_of_spec_2250": round(tflops / SPEC_BF16_TFLOPS, 4),
         "alone": alone,
+        "traffic": captured_traffic(w.name, "prefill", window, Hkv),
         "l2": "inputs exceed the 126 MB L2; launches back to back" if step.NL == 1 else
               f"{step.NL} copies of q, k, v and o ({step.NL * step.io_bytes / 1e6:.0f} MB in "
               f"all, above twice the 126 MB L2), launch i on copy i mod {step.NL}; launches "

@@ -43,6 +43,24 @@ def test_traffic_only_for_the_captured_configuration():
     assert bench.captured_traffic("no_such_workload", "decode", None, None) is None
     # the prefill capture is of the GQA shape; an MHA run (--hkv 32) has none
     assert bench.captured_traffic("swa_t32768", "prefill", 4096, 32) is None
+    # the ragged endpoints are captured separately
+    mqa = bench.captured_traffic("decode_ragged", "decode", None, 1)
+    mha = bench.captured_traffic("decode_ragged", "decode", None, 8)
+    assert mqa is not None and mha is not None and mha > 5 * mqa
+
+
+def test_captured_traffic_describes_the_current_kernels():
+    """Every recorded capture matches the kernels' current code (so the bench
+    reports it), and each is within 8 % above the launch's algorithmic bytes
+    (no wasted re-reads) -- the algorithmic bytes computed here from the
+    workload shapes."""
+    for e in bench.CAPTURED_TRAFFIC:
+        assert bench.captured_traffic(e["workload"], e["phase"], e["window"], e["hkv"]) == e["bytes"]
+    alg = {("decode_b8_n8000", None): 2 * 8 * 8 * 8001 * 128 * 2,
+           ("swa_t32768", None): 2 * 8 * 4096 * 128 * 2}
+    for (wl, hkv), b in alg.items():
+        got = bench.captured_traffic(wl, "decode", None, hkv)
+        assert b <= got <= 1.08 * b, (wl, got, b)
 
 
 def test_prefill_cpu_sample_rows_are_prefill_rows():
