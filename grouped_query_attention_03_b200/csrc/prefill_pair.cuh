@@ -19,15 +19,22 @@
 //               O_A += P_A(j) V_j, S_A(j+1), O_B += P_B(j) V_j, S_B(j+1)
 //               so the tensor pipe runs one head while the other head's
 //               softmax warps work.  P V takes P from TMEM (A operand) and
-//               V from shared memory; S(j+1) overwrites P(j) only after
-//               P V(j), since one thread's MMAs execute in issue order.
+//               V from shared memory, in two halves: keys 0-63 as soon as
+//               the softmax has written that half of P, then keys 64-127.
+//               S(j+1) overwrites P(j) only after P V(j), since one
+//               thread's MMAs execute in issue order; for the same reason
+//               S(j+1) being complete means P V(j) is, so the softmax never
+//               waits for P V separately.  Every wait of this thread comes
+//               before a group of MMAs: an MMA issue blocks while the
+//               tensor pipe's short queue is full.
 //   warps 2-3   idle (they complete the first warpgroup, which hands most of
 //               its registers to the softmax warpgroups with setmaxnreg).
 //   warps 4-7   softmax of head A, warps 8-11 softmax of head B: thread = row
 //               (TMEM lane); the whole 128-score row is read from TMEM into
 //               registers at once, then row max, lazy O rescale, and bf16 P
 //               written back to the same TMEM lane over the first 64 S
-//               columns (no shared-memory round trip for P); O / l epilogue.
+//               columns (no shared-memory round trip for P), its first half
+//               published on its own; O / l epilogue.
 // TMEM columns: S_A [0,128) (P_A in [0,64)), S_B [128,256) (P_B in
 // [128,192)), O_A [256, 256+d), O_B after it.  Shared memory holds the two
 // Q tiles and the K/V ring only.
@@ -97,7 +104,7 @@ __device__ __forceinline__ int row_lo(const Params &p, int b, int t) {
 struct Bars {
   uint64_t q_full;
   uint64_t full[kMaxSlots], empty[kMaxSlots];
-  uint64_t s_full[2], p_full[2], o_done[2];
+  uint64_t s_full[2], p_half[2], p_full[2], o_done[2];
   uint64_t mma_fin;
   uint64_t v_clean;  // the last V tile's rows past the sequence are zero
   uint32_t tmem_base;
@@ -123,7 +130,8 @@ __device__ __forceinline__ void rescale_o(uint32_t tO, float alpha) {
 // TMEM lane over the S columns it came from (column c holds p[2c], p[2c+1]),
 // where the P V MMA reads it as its A operand; returns the row sum.
 template <int D>
-__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP) {
+__device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint32_t tP,
+                                        uint64_t *half_bar) {
   float2 lsum2 = make_float2(0.f, 0.f);
   const float2 sc2 = make_float2(sc, sc), nm2 = make_float2(-m, -m);
 #pragma unroll
@@ -138,6 +146,12 @@ __device__ __forceinline__ float emit_p(const float *s, float sc, float m, uint3
       w[e] = __uint_as_float(pack_bf16(pv.x, pv.y));
     }
     tc::tmem_st32(tP + half * 32, w);
+    if (half == 0) {  // keys 0-63 of P: their P V can start
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      __syncwarp();
+      if ((threadIdx.x & 31) == 0) mbar_arrive(half_bar);
+    }
   }
   tc::tmem_wait_st();
   return lsum2.x + lsum2.y;
@@ -174,14 +188,8 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
 #pragma unroll
     for (int c = 0; c < kBN / 32; ++c) tc::tmem_ld32(tS + c * 32, s + c * 32);
     tc::tmem_wait_ld();
-    // O and P of this head are free once its previous PV has completed.
-    if (j >= 1) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (j - 1) & 1, failed))) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-    }
+    // O and P are free here: S(j) was committed after P V(j-1) by the same
+    // thread, so S(j) being ready means P V(j-1) has completed.
     if (edge) {
 #pragma unroll
       for (int i = 0; i < kBN; ++i) {
@@ -214,7 +222,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
       l_run *= alpha;
       m_run = m_new;
     }
-    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS);
+    const float lsum = emit_p<D>(s, sc, m_run == -INFINITY ? 0.f : m_run, tS, &bars.p_half[hd]);
     l_run += lsum;
     tc::fence_before_sync();
     __syncwarp();
@@ -224,7 +232,7 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
   // epilogue: O / l in bf16, one row per thread; the whole warp reads TMEM
   bool have = false;
   if (nt > 0 && ok) {
-    have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], (nt - 1) & 1, failed));
+    have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[hd], 0, failed));
     tc::fence_after_sync();
   }
   const float inv = (active && have && l_run > 0.f) ? 1.f / l_run : 0.f;
@@ -285,6 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&bars.s_full[h], 1);
+      mbar_init(&bars.p_half[h], 4);
       mbar_init(&bars.p_full[h], 4);
       mbar_init(&bars.o_done[h], 1);
     }
@@ -440,16 +449,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::mma_commit(&bars.s_full[hd]);
       };
-      auto issue_pv = [&](int hd, int j) {
-        // A = P from TMEM (over S of this head: 8 columns per 16 keys)
+      auto issue_pv = [&](int hd, int j, int k0) {
+        // A = P from TMEM (over S of this head: 8 columns per 16 keys);
+        // keys [16 k0, 16 k0 + 64)
         const uint32_t sV = slot_addr(2 * j + 1);
 #pragma unroll
-        for (int k = 0; k < kBN / 16; ++k) {
+        for (int k = k0; k < k0 + kBN / 32; ++k) {
           const uint64_t db = tc::sw128_desc(sV + k * 16 * 128, K::BLK, 1024);
           tc::mma_bf16_ts(tmem + K::TM_O + hd * D, tmem + hd * kBN + k * 8, db, idO,
                           (j > 0 || k > 0) ? 1u : 0u);
         }
-        tc::mma_commit(&bars.o_done[hd]);
       };
       bool ok = mbar_wait(&bars.q_full, 0, &failed) && wait_load(0);
       if (ok) {
@@ -459,26 +468,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_commit(&bars.empty[0]);  // K_0
       }
       for (int j = 0; ok && j < nt; ++j) {
-        // head A: O_A += P_A(j) V_j, then S_A(j+1)
-        if (!mbar_wait(&bars.p_full[0], j & 1, &failed) || !wait_load(2 * j + 1)) { ok = false; break; }
+        const bool more = j + 1 < nt;
+        // head A: first half of P V(j) once its keys 0-63 of P are written,
+        // then the second half and S_A(j+1)
+        if (!mbar_wait(&bars.p_half[0], j & 1, &failed) || !wait_load(2 * j + 1) ||
+            (more && !wait_load(2 * j + 2))) {
+          ok = false;
+          break;
+        }
         if (clear_v && j == nt - 1 && !mbar_wait(&bars.v_clean, 0, &failed)) { ok = false; break; }
         tc::fence_after_sync();
-        issue_pv(0, j);
-        if (j + 1 < nt) {
-          if (!wait_load(2 * j + 2)) { ok = false; break; }
-          tc::fence_after_sync();
-          issue_s(0, j + 1);
-        }
-        // head B: O_B += P_B(j) V_j (frees V_j), then S_B(j+1) (frees K_j+1)
+        issue_pv(0, j, 0);
+        if (!mbar_wait(&bars.p_full[0], j & 1, &failed)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(0, j, 4);
+        if (more) issue_s(0, j + 1);
+        // head B likewise; then V_j and K_(j+1) are free
+        if (!mbar_wait(&bars.p_half[1], j & 1, &failed)) { ok = false; break; }
+        tc::fence_after_sync();
+        issue_pv(1, j, 0);
         if (!mbar_wait(&bars.p_full[1], j & 1, &failed)) { ok = false; break; }
         tc::fence_after_sync();
-        issue_pv(1, j);
+        issue_pv(1, j, 4);
         tc::mma_commit(&bars.empty[(2 * j + 1) % K::NSLOT]);
-        if (j + 1 < nt) {
+        if (more) {
           issue_s(1, j + 1);
           tc::mma_commit(&bars.empty[(2 * j + 2) % K::NSLOT]);
         }
       }
+      tc::mma_commit(&bars.o_done[0]);  // O_A and O_B complete (read by the epilogue)
+      tc::mma_commit(&bars.o_done[1]);
       // Drain: every MMA this thread issued has finished before TMEM is freed.
       tc::mma_commit(&bars.mma_fin);
       bool f2 = false;
