@@ -170,6 +170,8 @@ DECODE_SOURCES = ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"]
 DECODE_SHA = "b36d81a54f38f0e6833eb54afe7b30de32d3c5f26ca7ac64b09690ae6d3fce86"
 PAIR_SOURCES = ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"]
 PAIR_SHA = "d334ae112e55900a4675c19d3a5e120f6ede0e0814cf43e52814b6296a4d8535"
+SPLIT_SOURCES = ["prefill_split.cuh", "common.cuh", "tc_ptx.cuh"]
+SPLIT_SHA = "ba5ade7553d65e90021c9814939ad7640c7124a3dc89340fefc6d13982c448df"
 CAPTURED_TRAFFIC = [
     {"workload": "decode_b8_n8000", "phase": "decode", "window": None, "hkv": None,
      "bytes": 267_997_440, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
@@ -180,9 +182,13 @@ CAPTURED_TRAFFIC = [
     {"workload": "swa_t32768", "phase": "decode", "window": None, "hkv": None,
      "bytes": 17_122_304, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": None, "hkv": None,
-     "bytes": 6_351_104, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 6_523_136, "sources": SPLIT_SOURCES, "sha256": SPLIT_SHA},
+    {"workload": "prefill_b4_t1024", "phase": "prefill", "window": 256, "hkv": None,
+     "bytes": 6_350_848, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": None,
      "bytes": 686_371_840, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+    {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": 32,
+     "bytes": 1_059_718_656, "sources": SPLIT_SOURCES, "sha256": SPLIT_SHA},
 ]
 
 
@@ -623,10 +629,15 @@ class PrefillStep:
     def kernel(self):
         """The tensor-core kernel gqa_prefill dispatches to for this shape."""
         w = self.w
-        if w.d in (64, 128) and (w.Hq // self.Hkv) % 2 == 0:
-            return "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)"
-        return ("pfs::prefill_split_kernel (one query head per CTA, two softmax warpgroups "
-                "of 64 score columns each)")
+        return self.gqa.prefill_kernel(w.B, w.Hq, self.Hkv, w.T, w.d, self.window)
+
+
+KERNEL_NAMES = {
+    "simt": "prefill_simt_kernel (CUDA cores)",
+    "pair": "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)",
+    "split": "pfs::prefill_split_kernel (one query head per CTA; two softmax warpgroups over "
+           "keys 0-63 and 64-127 of each tile, each with its own running maximum, sum and O)",
+}
 
 
 def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PASSES):
@@ -669,7 +680,7 @@ def measure_prefill(w, window, device, reps, warmup, Hkv=None, min_passes=MIN_PA
     sustained = sum(ms_pass) > 250.0 and "bf16_tflops_sustained" in peaks
     peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     res = {
-        **step.describe(), "kernel": step.kernel(), "tflops": round(tflops, 2), "ms": round(ms, 5),
+        **step.describe(), "kernel": KERNEL_NAMES[step.kernel()], "tflops": round(tflops, 2), "ms": round(ms, 5),
         "launches_per_pass": reps, "passes": st["passes"],
         "pass_ms": {k: round(v, 5) for k, v in st.items() if k != "passes"},
         "timed_ms": round(sum(ms_pass), 2),
@@ -925,7 +936,7 @@ def run_gpu_prefill(args, world, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded normal rounded to bf16)",
         "config": dict(step.describe(), parallelism=f"replicas x{world}", l2=res["l2"]),
-        "roofline": {"bound": "tensor", "kernel": step.kernel(),
+        "roofline": {"bound": "tensor", "kernel": KERNEL_NAMES[step.kernel()],
                      "achieved": res["tflops"], "peak": res["peak"],
                      "peak_kind": res["peak_kind"], "unit": "TFLOP/s",
                      "frac": res["frac_of_measured"], "frac_of_burst": res["frac_of_burst"],

@@ -45,6 +45,21 @@ struct DeviceInfo {
   int major = 0;
 };
 
+// The paired prefill kernel's grid for a plain prompt leaves SMs idle and
+// its longest query tile (the last one) walks more than 4 KV tiles: one
+// head per CTA is faster there (see the dispatch in attend_impl).
+bool prefill_prefers_split(int B, int Hq, int Hkv, int Tq, int Tk, int cached, bool seg,
+                           int window, int sms) {
+  if (cached || seg || Tq != Tk || Tq <= 0) return false;
+  const long long num_mt = (Tq + 127) / 128;
+  const long long pair_grid = (long long)B * Hkv * ((Hq / Hkv) / 2) * num_mt;
+  if (pair_grid >= sms) return false;
+  const long long a0 = (num_mt - 1) * 128;
+  const long long hi = Tq - 1;
+  const long long lo = window > 0 ? std::max(0LL, a0 - (window - 1)) : 0;
+  return hi / 128 - lo / 128 + 1 > 4;
+}
+
 gqa_status device_info(DeviceInfo *out) {
   static std::mutex mu;
   static DeviceInfo cache[64];
@@ -294,6 +309,17 @@ int gqa_kv_head_for_query(int h, int Hq, int Hkv) {
   return h / (Hq / Hkv);
 }
 
+int gqa_prefill_kernel(int B, int Hq, int Hkv, int T, int d, int window, int sms) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || sms <= 0 || Hq % Hkv != 0)
+    return -1;
+  if (window == 0 || window < -1) return -1;
+  if (!gqa::pfs::supported(d)) return 0;
+  if (gqa::pf2::supported(d, Hq, Hkv) &&
+      !prefill_prefers_split(B, Hq, Hkv, T, T, 0, false, window, sms))
+    return 1;
+  return 2;
+}
+
 int gqa_window_start(int t, int window) {
   if (t < 0 || window == 0 || window < -1) return -1;
   if (window < 0) return 0;
@@ -347,8 +373,14 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
       aligned16(k) && aligned16(v) && aligned16(o)) {
     // Heads of a group in pairs (one CTA per pair, each K/V tile fetched
     // once for both) when the group size is even; otherwise one head per
-    // CTA, its score rows split over two softmax warpgroups.
-    if (gqa::pf2::supported(d, Hq, Hkv))
+    // CTA, its key tiles split over two softmax warpgroups.  A plain prompt
+    // whose paired grid leaves SMs idle and whose longest query tile walks
+    // more than 4 KV tiles also takes one head per CTA: there the longest
+    // CTA's chain sets the time, and a head's tile costs about half a pair's
+    // (measured: B=4, Hq=8, Hkv=2, d=64, T=1024 causal 17.5 against 21.6 us;
+    // with a 256-key window, 3 tiles, the pair stays faster, 13.6 against 17.3).
+    if (gqa::pf2::supported(d, Hq, Hkv) &&
+        !(prefill_prefers_split(B, Hq, Hkv, Tq, Tk, cached, seg != nullptr, window, di.sms)))
       return gqa::pf2::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached,
                               d, window, scale_log2, dev_status, st);
     return gqa::pfs::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,

@@ -1,6 +1,6 @@
 // prefill_split.cuh -- tcgen05/TMEM causal-windowed GQA prefill, one query
-// head per CTA, each score row shared by two softmax warpgroups (bf16,
-// sm_100a).
+// head per CTA, each 128-key tile's scores shared by two softmax warpgroups
+// that each keep their own running maximum, sum and O (bf16, sm_100a).
 //
 // What it computes ("Share key/value heads and make context explicit",
 // sections "Give each query head an explicit shared KV head" and "Intersect
@@ -8,33 +8,36 @@
 // max/sum from "GQA, FlashAttention and the KV cache"): for every batch row
 // b, query head h and active cell t < n_b, softmax over the permitted keys
 // of scale * q.k, mixed with the value rows of the shared lane g(h);
-// inactive rows are zero.  It serves group sizes the paired kernel
-// (prefill_pair.cuh) cannot: odd ones, MHA included.
+// inactive rows are zero.  It serves odd group sizes (MHA included), which
+// the paired kernel (prefill_pair.cuh) cannot, and short prompts whose
+// paired grid would leave SMs idle.
 //
 // One CTA owns a 128-row query tile of one (b, h) and walks the 128-key
 // tiles that intersect its permitted band, skipping tiles wholly outside
-// the causal window.  The two halves of every 128-score row belong to two
-// warpgroups, so a KV tile's softmax takes about half as long as with one
-// thread per whole row, and both S and P are double-buffered in TMEM, so
-// the softmax of tile j runs while the tensor cores compute S(j+1) and
-// P V(j-1), and waits for them only to rescale O:
+// the causal window.  Keys 0-63 of every tile belong to one softmax
+// warpgroup and keys 64-127 to the other.  Each runs the online softmax
+// over its own keys only (its own running maximum and sum) and accumulates
+// its own O_h = sum P_h V_h, so the two never wait for each other inside
+// the loop; the epilogue combines them once:
+//   O = (O_0 a_0 + O_1 a_1) / (l_0 a_0 + l_1 a_1),  a_h = 2^(m_h - max(m_0, m_1)),
+// the same merge as two split-K partials.  S is double-buffered in TMEM, so
+// the softmax of tile j runs while the tensor cores compute S(j+1):
 //   warp 0      TMA producer: Q once, then K and V tiles into 2-stage rings
 //               (128-byte swizzle, no multicast).
 //   warp 1      allocates TMEM; lane 0 issues tcgen05.mma: S(j) = Q K_j^T
-//               into S[j%2] (M=N=128, K=d), then O += P(j-1) V_{j-1}
-//               (M=128, N=d, K=128, P read from TMEM as the A operand).
+//               into S[j%2] (M=N=128, K=d), then for each key half h once
+//               its P is written, O_h += P_h(j-1) V_{j-1}[64h, 64h+64)
+//               (M=128, N=d, K=64, P read from TMEM as the A operand).
 //   warps 2-3   idle (they complete the first warpgroup, which hands most of
 //               its registers to the softmax warpgroups with setmaxnreg).
-//   warps 4-7   softmax of score columns 0-63, warps 8-11 of columns 64-127:
-//               thread = query row (TMEM lane).  Per tile each half takes its
-//               64 scores, masks edge tiles, posts its maximum in shared
-//               memory and waits (bounded, on x_full) for the other half's,
-//               rescales its half of O when the row maximum grew by more than
-//               2^8 (lazy rescale), and writes its 32 columns of bf16 P; the
-//               two halves' row sums are added in the epilogue, where each
-//               half writes its d/2 columns of O / l.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+d), P0 and P1 (bf16,
-// two keys per 32-bit column) [256+d, 320+d) and [320+d, 384+d).
+//   warps 4-7   softmax of keys 0-63, warps 8-11 of keys 64-127: thread =
+//               query row (TMEM lane).  Per tile each half takes its 64
+//               scores, masks edge tiles, rescales its O when its maximum
+//               grew by more than 2^8 (lazy rescale), and writes 32 columns
+//               of bf16 P over the first half of its own S columns.
+// TMEM columns: S0 [0,128), S1 [128,256), O_0 [256, 256+d), O_1 [256+d,
+// 256+2d); P_h(j) over S[j%2] columns [64h, 64h+32).  S(j) overwrites P(j-2)
+// only after P V(j-2), which the same thread issued first.
 #pragma once
 
 #include <cuda.h>
@@ -54,6 +57,8 @@ constexpr int kRegsLow = 72, kRegsHigh = 216;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Query tiles per head from which CTAs are ordered head by head.
+constexpr int kHeadMajorTiles = 64;
 
 template <int D>
 struct Cfg {
@@ -65,9 +70,8 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + TILE;
   static constexpr int OFF_V = OFF_K + STAGES * TILE;
   static constexpr int DYN_BYTES = OFF_V + STAGES * TILE;
-  static constexpr uint32_t TM_O = 256;
-  static constexpr uint32_t TM_P = 256 + D;         // P0; P1 = TM_P + 64
-  static_assert(TM_P + kBN <= kTmemCols, "S, O and two P buffers must fit in TMEM");
+  static constexpr uint32_t TM_O = 256;              // O of key half 0; half 1 at TM_O + D
+  static_assert(TM_O + 2 * D <= kTmemCols, "two S buffers and two O halves must fit in TMEM");
   // At least 120 KB so that only one CTA (which holds all 512 TMEM columns)
   // is resident per SM.
   static constexpr int SMEM = (DYN_BYTES + 1024 > 120 * 1024 ? DYN_BYTES + 1024 : 120 * 1024);
@@ -85,6 +89,7 @@ struct Params {
   const int32_t *seg;  // prompt only: [B,Tq] first key cell of row t's
                        // packed segment, or NULL (segment start 0)
   float scale_log2;
+  int head_major;  // CTA order: 1 head by head, 0 query tile by query tile
 };
 
 // First permitted key of query position t ("Intersect the window with the
@@ -102,9 +107,9 @@ __device__ __forceinline__ int row_lo(const Params &p, int b, int t) {
 struct Bars {
   uint64_t q_full;
   uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
-  uint64_t s_full[2], s_free[2];  // S[s] written by the MMA / read by the softmax
-  uint64_t p_full[2], o_done[2];  // P[s] written / P V of a P[s] tile complete
-  uint64_t x_full;                // both halves posted their value
+  uint64_t s_full[2];             // S[s] written by the MMA
+  uint64_t p_full[2][2];          // [s][half]: that half's P written over S[s]
+  uint64_t o_done[2];             // both halves' P V of an S[s] tile complete
   uint64_t mma_fin;
   uint32_t tmem_base;
 };
@@ -117,15 +122,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   using K = Cfg<D>;
   extern __shared__ unsigned char smem_raw[];
   __shared__ Bars bars;
-  __shared__ float xbuf[2 * 2 * kBM];  // [exchange parity][half][row]
+  __shared__ float xbuf[2 * 2 * kBM];  // [m, l][half][row], exchanged once at the end
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- which tile: longest causal rows first; heads of a KV group adjacent
+  // ---- which tile.  Short prompts: longest causal rows first over all
+  // heads (the longest CTAs start in the first wave).  Long ones (head_major):
+  // head by head, its query tiles from the last, so the CTAs in flight share
+  // a few heads' K/V windows in L2 instead of one tile of every head.
   const int BH = p.B * p.Hq;
-  const int mt = p.num_mt - 1 - (int)(blockIdx.x / BH);
-  const int bh = (int)(blockIdx.x % BH);
+  int mt, bh;
+  if (p.head_major) {
+    bh = (int)(blockIdx.x / p.num_mt);
+    mt = p.num_mt - 1 - (int)(blockIdx.x % p.num_mt);
+  } else {
+    mt = p.num_mt - 1 - (int)(blockIdx.x / BH);
+    bh = (int)(blockIdx.x % BH);
+  }
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int m0 = mt * kBM;
@@ -138,11 +152,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.k_empty[s], 1);
       mbar_init(&bars.v_empty[s], 1);
       mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.s_free[s], 8);  // every softmax warp
-      mbar_init(&bars.p_full[s], 8);
+      mbar_init(&bars.p_full[s][0], 4);  // the half's four warps
+      mbar_init(&bars.p_full[s][1], 4);
       mbar_init(&bars.o_done[s], 1);
     }
-    mbar_init(&bars.x_full, 8);
     mbar_init(&bars.mma_fin, 1);
     fence_mbar_init();
   }
@@ -226,25 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool active = t < off + rows;
     const int lo_t = active ? row_lo(p, b, t) : 0;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    const uint32_t tO = tmem + lane_base + K::TM_O + half * (D / 2);
+    const uint32_t tO = tmem + lane_base + K::TM_O + half * D;  // this half's O
     const float sc = p.scale_log2;
+    // Each half keeps its own running maximum and sum over its 64 keys of
+    // every tile and its own O; the two are combined once, in the epilogue.
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int xn = 0;  // exchanges so far: the phase of x_full
-    // Post v for the other half of the same rows, wait (bounded) for its
-    // value; the arrive/wait pair also orders both halves' TMEM reads.
-    auto exchange = [&](float v, float *other) -> bool {
-      float *slot = xbuf + (xn & 1) * 2 * kBM;
-      slot[half * kBM + row] = v;
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.x_full);
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&bars.x_full, xn & 1, &failed)) != 0;
-      tc::fence_after_sync();
-      xn++;
-      *other = slot[(1 - half) * kBM + row];
-      return got;
-    };
     for (int j = 0; j < nt; ++j) {
       const int sb = j & 1;
       const int kt = (j0 + j) * kBN;     // key of the tile's first column
@@ -254,14 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc::fence_after_sync();
+      const uint32_t tS = tmem + lane_base + sb * kBN + half * 64;
       float s[64];
-      tc::tmem_ld32(tmem + lane_base + sb * kBN + half * 64, s);
-      tc::tmem_ld32(tmem + lane_base + sb * kBN + half * 64 + 32, s + 32);
+      tc::tmem_ld32(tS, s);
+      tc::tmem_ld32(tS + 32, s + 32);
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.s_free[sb]);
-
       const bool edge = (kb + 63 > a0) || (kb < lo_max);
       if (edge) {
 #pragma unroll
@@ -270,8 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (key > t || key < lo_t) s[c] = -INFINITY;
         }
       }
-      // this half's maximum of s*scale (sc*max(s) for sc > 0, sc*min(s)
-      // otherwise), then the row's over both halves
+      // this half's maximum of s*scale (sc*max(s) for sc > 0, sc*min(s) otherwise)
       float mx;
       {
         const bool neg = !(sc > 0.f);
@@ -286,20 +282,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mx = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
       }
-      const float m_half = (mx == -INFINITY) ? -INFINITY : mx * fabsf(sc);
-      float m_other;
-      if (!exchange(m_half, &m_other)) {
-        ok = false;
-        break;
-      }
-      const float m_tile = fmaxf(m_half, m_other);
+      const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * fabsf(sc);
       if (j == 0) {
         m_run = m_tile;
       } else if (__any_sync(0xffffffffu, m_tile > m_run + kRescaleThreshold)) {
-        // O must hold P V(j-1) before it is rescaled: o_done[(j-1)%2]
-        // completes its ((j-1)/2)-th phase with it (it cannot be two phases
-        // further: P(j+1) is not written yet).  The warps of both halves
-        // over the same rows take the same decision.
+        // This half's O must hold P V(j-1) before it is rescaled: o_done of
+        // S[(j-1)%2] completes its ((j-1)/2)-th phase with it.  P(j) itself
+        // needs no wait: S(j) was issued after P V(j-2) by the same thread,
+        // so S(j) ready means P V(j-2) has read the P that P(j) overwrites.
         const int pj = j - 1;
         if (!__all_sync(0xffffffffu,
                         mbar_wait(&bars.o_done[pj & 1], (pj >> 1) & 1, &failed))) {
@@ -310,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = m_new == m_run ? 1.f : exp2f(m_run - m_new);  // 0 from -inf
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 32; ++c) {
           float ov[32];
           tc::tmem_ld32(tO + c * 32, ov);
           tc::tmem_wait_ld();
@@ -322,16 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run *= alpha;
         m_run = m_new;
       }
-      // P(j) goes to P[sb], which P V(j-2) read: o_done[sb] completes its
-      // ((j-2)/2)-th phase with that MMA.
-      if (j >= 2) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.o_done[sb], ((j - 2) >> 1) & 1, &failed))) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-      }
-      // bf16 P into this thread's TMEM lane (column c of this half holds
+      // bf16 P over the first 32 of this half's S columns (column c holds
       // p[2c], p[2c+1]), where the P V MMA reads it as its A operand.
       {
         const float msub = m_run == -INFINITY ? 0.f : m_run;
@@ -345,19 +326,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           lsum2 = fadd2v(lsum2, pv);
           w[e] = __uint_as_float(pack_bf16(pv.x, pv.y));
         }
-        tc::tmem_st32(tmem + lane_base + K::TM_P + sb * 64 + half * 32, w);
+        tc::tmem_st32(tS, w);
         tc::tmem_wait_st();
         l_run += lsum2.x + lsum2.y;
       }
-      if (half == 0 && kt + kBN > n_keys) {
+      if (kt + kBN > n_keys && (row >> 6) == half) {
         // Cells past the sequence in this V tile are not the sequence's (an
         // unwritten cache cell may hold NaN): their p is 0, but 0 * NaN is
-        // not, so clear those rows (thread = row) before P V is issued.
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.v_full[sb], (j >> 1) & 1, &failed))) {
-          ok = false;
-          break;
-        }
-        if (kt + row >= n_keys) {
+        // not, so clear those rows before P V is issued.  V row r is cleared
+        // by thread r of the half whose keys it holds (rows 0-63: half 0).
+        bool vok = mbar_wait(&bars.v_full[sb], (j >> 1) & 1, &failed);
+        if (vok && kt + row >= n_keys) {
           unsigned char *vrow = smem + K::OFF_V + sb * K::TILE + row * 128;
 #pragma unroll
           for (int c = 0; c < K::KB; ++c)
@@ -366,46 +345,60 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4 *>(vrow + c * K::BLK + ch * 16) = make_uint4(0, 0, 0, 0);
         }
         tc::fence_proxy_async_smem();
+        if (!__all_sync(0xffffffffu, vok)) {
+          ok = false;
+          break;
+        }
       }
       tc::fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.p_full[sb]);
+      if (lane == 0) mbar_arrive(&bars.p_full[sb][half]);
     }
 
-    // ---- epilogue: O / l in bf16 over this half's d/2 columns, one row per
-    // thread (the whole warp reads TMEM; only rows inside the tensor are
-    // stored).  The last P V completes the last phase of o_done[(nt-1)%2],
-    // after every earlier MMA of the issuing thread.
+    // ---- epilogue.  The last P V of both halves completes the last phase
+    // of o_done[(nt-1)%2] (after every earlier MMA of the issuing thread).
+    // The halves swap their (maximum, sum) once through shared memory, then
+    // each writes d/2 columns of O = (O_0 a_0 + O_1 a_1) / (l_0 a_0 + l_1 a_1),
+    // a_h = 2^(m_h - max(m_0, m_1)), one row per thread.
     bool have = false;
     if (nt > 0 && ok) {
       const int lj = nt - 1;
       have = __all_sync(0xffffffffu, mbar_wait(&bars.o_done[lj & 1], (lj >> 1) & 1, &failed));
       tc::fence_after_sync();
     }
-    float l_other = 0.f;
-    if (have) have = exchange(l_run, &l_other);
-    const float l_row = l_run + l_other;
+    xbuf[half * kBM + row] = m_run;
+    xbuf[2 * kBM + half * kBM + row] = l_run;
+    asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight softmax warps
+    const float m_o = xbuf[(1 - half) * kBM + row];
+    const float l_o = xbuf[2 * kBM + (1 - half) * kBM + row];
+    const float m_all = fmaxf(m_run, m_o);
+    const float a_me = m_all == -INFINITY ? 0.f : exp2f(m_run - m_all);
+    const float a_o = m_all == -INFINITY ? 0.f : exp2f(m_o - m_all);
+    const float l_row = l_run * a_me + l_o * a_o;
     const float inv = (active && have && l_row > 0.f) ? 1.f / l_row : 0.f;
+    // output columns [half * d/2, half * d/2 + d/2): this half's O and the other's
+    const uint32_t tOa = tmem + lane_base + K::TM_O + half * (D / 2);        // O_0 columns
+    const uint32_t tOb = tmem + lane_base + K::TM_O + D + half * (D / 2);    // O_1 columns
+    const float c0 = half == 0 ? a_me : a_o, c1 = half == 0 ? a_o : a_me;
     __nv_bfloat16 *orow =
         p.o + (((size_t)b * p.Hq + h) * p.Tq + min(qr, p.Tq - 1)) * D + half * (D / 2);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
-      float ov[32];
+      float ov[32], ow[32];
       if (have) {
-        tc::tmem_ld32(tO + c * 32, ov);
+        tc::tmem_ld32(tOa + c * 32, ov);
+        tc::tmem_ld32(tOb + c * 32, ow);
         tc::tmem_wait_ld();
       }
-      if (!have || !active) {  // inactive rows are exact zeros (their O may be NaN)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ov[i] = 0.f;
-      }
+      for (int i = 0; i < 32; ++i)  // inactive rows are exact zeros (their O may be NaN)
+        ov[i] = (have && active) ? (ov[i] * c0 + ow[i] * c1) * inv : 0.f;
       if (qr < p.Tq) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           uint32_t w4[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w4[i] = pack_bf16(ov[e * 8 + 2 * i] * inv, ov[e * 8 + 2 * i + 1] * inv);
+          for (int i = 0; i < 4; ++i) w4[i] = pack_bf16(ov[e * 8 + 2 * i], ov[e * 8 + 2 * i + 1]);
           *reinterpret_cast<uint4 *>(orow + c * 32 + e * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
@@ -457,19 +450,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idS = tc::idesc_bf16_f32(kBM, kBN, 0, 0);
         constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
         const uint32_t sQ = smem_u32(smem + K::OFF_Q);
-        // O += P(i) V_i: P from P[i%2] once both halves wrote it, V from its
-        // ring stage; commits o_done[i%2] (its (i/2)-th phase) and frees V.
+        // O_h += P_h(i) V_i[64h, 64h+64) for key half h: P_h over the first
+        // 32 columns of that half of S[i%2], once that half has written it;
+        // V from its ring stage.  Commits o_done[i%2] (its (i/2)-th phase)
+        // and frees V.
         auto issue_pv = [&](int i) -> bool {
           const int s = i & 1;
-          if (!mbar_wait(&bars.p_full[s], (i >> 1) & 1, &failed)) return false;
           if (!mbar_wait(&bars.v_full[s], (i >> 1) & 1, &failed)) return false;
-          tc::fence_after_sync();
           const uint32_t sV = smem_u32(smem + K::OFF_V + s * K::TILE);
 #pragma unroll
-          for (int k = 0; k < kBN / 16; ++k) {  // A = P from TMEM, 8 columns per 16 keys
-            const uint64_t db = tc::sw128_desc(sV + k * 16 * 128, K::BLK, 1024);
-            tc::mma_bf16_ts(tmem + K::TM_O, tmem + K::TM_P + s * 64 + k * 8, db, idO,
-                            (i > 0 || k > 0) ? 1u : 0u);
+          for (int hh = 0; hh < 2; ++hh) {
+            if (!mbar_wait(&bars.p_full[s][hh], (i >> 1) & 1, &failed)) return false;
+            tc::fence_after_sync();
+#pragma unroll
+            for (int k = 4 * hh; k < 4 * hh + 4; ++k) {  // A = P from TMEM, 8 columns per 16 keys
+              const uint64_t db = tc::sw128_desc(sV + k * 16 * 128, K::BLK, 1024);
+              tc::mma_bf16_ts(tmem + K::TM_O + hh * D, tmem + s * kBN + hh * 64 + (k - 4 * hh) * 8,
+                              db, idO, (i > 0 || k > 4 * hh) ? 1u : 0u);
+            }
           }
           tc::mma_commit(&bars.o_done[s]);
           tc::mma_commit(&bars.v_empty[s]);
@@ -478,8 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = mbar_wait(&bars.q_full, 0, &failed);
         for (int j = 0; ok && j < nt; ++j) {
           const int sb = j & 1;
-          // S[sb] was read by the softmax of tile j-2 (its (j/2 - 1)-th phase)
-          if (j >= 2 && !mbar_wait(&bars.s_free[sb], ((j >> 1) - 1) & 1, &failed)) break;
+          // S(j) overwrites P(j-2) in S[sb]: P V(j-2) was issued before it.
           if (!mbar_wait(&bars.k_full[sb], (j >> 1) & 1, &failed)) break;
           tc::fence_after_sync();
           const uint32_t sK = smem_u32(smem + K::OFF_K + sb * K::TILE);
@@ -550,6 +547,7 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.window = window;
   p.num_mt = (Tq + kBM - 1) / kBM;
   p.scale_log2 = scale_log2;
+  p.head_major = p.num_mt >= kHeadMajorTiles;
   const long long grid = (long long)B * Hq * p.num_mt;
   if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
   if (launch_dependent(prefill_split_kernel<D>, dim3((unsigned)grid), dim3(kThreads), K::SMEM,

@@ -28,7 +28,7 @@ STATUS_NAMES = {
 # Every symbol include/gqa.h declares.
 EXPORTS = ("gqa_prefill", "gqa_prefill_packed", "gqa_decode", "gqa_decode_workspace_bytes",
            "gqa_decode_append", "gqa_decode_multi", "gqa_decode_noalloc", "gqa_cache_append", "gqa_cache_bytes",
-           "gqa_ring_append", "gqa_ring_decode_append", "gqa_kv_head_for_query", "gqa_window_start", "gqa_status_string",
+           "gqa_ring_append", "gqa_ring_decode_append", "gqa_kv_head_for_query", "gqa_window_start", "gqa_prefill_kernel", "gqa_status_string",
            "gqa_version", "gqa_selftest_wait_timeout")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # GQA_NOALLOC_SCRATCH_BYTES in include/gqa.h
@@ -83,6 +83,8 @@ def _declare(L):
     L.gqa_cache_bytes.restype = ctypes.c_uint64
     L.gqa_kv_head_for_query.argtypes = [i32] * 3
     L.gqa_kv_head_for_query.restype = i32
+    L.gqa_prefill_kernel.argtypes = [i32] * 7
+    L.gqa_prefill_kernel.restype = i32
     L.gqa_window_start.argtypes = [i32, i32]
     L.gqa_window_start.restype = i32
     L.gqa_status_string.argtypes = [i32]
@@ -382,6 +384,18 @@ def cache_append(k_cache, v_cache, k_new, v_new, seq_lens, *, status=None, strea
 
 def cache_bytes(L, B, T, Hkv, d, elem_bytes):
     return int(lib().gqa_cache_bytes(L, B, T, Hkv, d, elem_bytes))
+
+
+def prefill_kernel(B, Hq, Hkv, T, d, window=None, sms=None):
+    """Which kernel gqa_prefill runs for a bf16 prompt of this shape: "pair"
+    (two heads of a KV group per CTA), "split" (one head per CTA) or "simt"
+    (CUDA cores).  `sms` defaults to the current device's SM count."""
+    if sms is None:
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    r = lib().gqa_prefill_kernel(B, Hq, Hkv, T, d, -1 if window is None else window, sms)
+    if r < 0:
+        raise ValueError(f"prefill_kernel: invalid arguments {(B, Hq, Hkv, T, d, window, sms)}")
+    return ("simt", "pair", "split")[r]
 
 
 def kv_head_for_query(h, Hq, Hkv):

@@ -325,6 +325,19 @@ uint64_t gqa_cache_bytes(int64_t L, int64_t B, int64_t T, int64_t Hkv,
  * not positive, Hq % Hkv != 0, or h is outside [0, Hq). */
 int gqa_kv_head_for_query(int h, int Hq, int Hkv);
 
+/* Which tensor-core kernel gqa_prefill runs for a bf16 prompt (no packed
+ * segments, 16-byte-aligned tensors) of B x Hq query heads over Hkv KV heads,
+ * T cells, head width d and window (GQA_NO_WINDOW or w >= 1) on a device with
+ * `sms` SMs:
+ *   1  two query heads of one KV group per CTA (even group size), unless:
+ *   2  one query head per CTA, its keys split over two softmax warpgroups
+ *      (odd group size; or a prompt whose paired grid has fewer CTAs than
+ *      `sms` and whose last query tile walks more than 4 KV tiles);
+ *   0  the CUDA-core kernel (d other than 64 or 128);
+ *  -1  invalid arguments (non-positive sizes, Hq % Hkv != 0, bad window).
+ * Host-only: reads nothing on the device and launches nothing. */
+int gqa_prefill_kernel(int B, int Hq, int Hkv, int T, int d, int window, int sms);
+
 /* [P1] causal_window_start with segment start 0: the first permitted key
  * cell of query cell t, max(0, t - (w-1)) (0 for GQA_NO_WINDOW); -1 for an
  * invalid window or t < 0. */

@@ -257,3 +257,20 @@ def test_selftest_wait_host_refusals(L):
     assert L.gqa_selftest_wait_timeout(2000001, 0, fake, fake, None) == SHAPE
     assert L.gqa_selftest_wait_timeout(1000, 0, None, fake, None) == NULL
     assert L.gqa_selftest_wait_timeout(1000, 0, fake, None, None) == NULL
+
+
+def test_prefill_kernel_choice(L):
+    """gqa_prefill_kernel names the kernel gqa_prefill runs (host-only)."""
+    pick = lambda B, Hq, Hkv, T, d, w, sms=148: L.gqa_prefill_kernel(B, Hq, Hkv, T, d, w, sms)
+    assert pick(1, 32, 8, 32768, 128, 4096) == 1   # even group, many CTAs: paired heads
+    assert pick(1, 32, 32, 32768, 128, 4096) == 2  # MHA (group of 1): one head per CTA
+    assert pick(1, 12, 4, 4096, 64, -1) == 2       # group of 3
+    assert pick(4, 8, 2, 1024, 64, -1) == 2        # 128 paired CTAs, last tile walks 8 KV tiles
+    assert pick(4, 8, 2, 1024, 64, 256) == 1       # ... with a 256 window only 3
+    assert pick(4, 8, 2, 1024, 64, -1, sms=64) == 1  # the paired grid fills the device
+    assert pick(4, 8, 2, 512, 64, -1) == 1         # 4 query tiles: the last walks 4 KV tiles
+    assert pick(4, 8, 2, 513, 64, -1) == 2         # 5 query tiles, the last walks 5
+    assert pick(1, 8, 2, 1024, 96, -1) == 0        # head width without a tensor-core kernel
+    for bad in ((0, 8, 2, 64, 64, -1), (1, 8, 3, 64, 64, -1), (1, 8, 2, 64, 64, 0),
+                (1, 8, 2, 64, 64, -2), (1, 8, 2, 0, 64, -1), (1, 8, 2, 64, 64, -1, 0)):
+        assert pick(*bad) == -1, bad

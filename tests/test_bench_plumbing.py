@@ -41,8 +41,11 @@ def test_traffic_only_for_the_captured_configuration():
     assert bench.captured_traffic("decode_b8_n8000", "decode", 512, None) is None
     assert bench.captured_traffic("decode_b8_n8000", "decode", None, 1) is None
     assert bench.captured_traffic("no_such_workload", "decode", None, None) is None
-    # the prefill capture is of the GQA shape; an MHA run (--hkv 32) has none
-    assert bench.captured_traffic("swa_t32768", "prefill", 4096, 32) is None
+    # the GQA and MHA prefills are captured separately (different kernels)
+    gqa_pf = bench.captured_traffic("swa_t32768", "prefill", 4096, None)
+    mha_pf = bench.captured_traffic("swa_t32768", "prefill", 4096, 32)
+    assert gqa_pf is not None and mha_pf is not None and mha_pf > gqa_pf
+    assert bench.captured_traffic("swa_t32768", "prefill", 4096, 16) is None
     # the ragged endpoints are captured separately
     mqa = bench.captured_traffic("decode_ragged", "decode", None, 1)
     mha = bench.captured_traffic("decode_ragged", "decode", None, 8)
@@ -61,6 +64,15 @@ def test_captured_traffic_describes_the_current_kernels():
     for (wl, hkv), b in alg.items():
         got = bench.captured_traffic(wl, "decode", None, hkv)
         assert b <= got <= 1.08 * b, (wl, got, b)
+    # prefill: q, k and v are read once (o may still sit in L2 at the end)
+    MB = 1 << 20
+    pf_in = {("prefill_b4_t1024", None, None): 4 * (8 + 2 + 2) * 1024 * 64 * 2,
+             ("prefill_b4_t1024", 256, None): 4 * (8 + 2 + 2) * 1024 * 64 * 2,
+             ("swa_t32768", 4096, None): (32 + 8 + 8) * 32768 * 128 * 2,
+             ("swa_t32768", 4096, 32): (32 + 32 + 32) * 32768 * 128 * 2}
+    for (wl, win, hkv), b in pf_in.items():
+        got = bench.captured_traffic(wl, "prefill", win, hkv)
+        assert b <= got <= 1.08 * (b + (32 * 32768 * 128 * 2 if wl == "swa_t32768" else 0)) + MB, (wl, got, b)
 
 
 def test_prefill_cpu_sample_rows_are_prefill_rows():
