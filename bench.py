@@ -170,8 +170,8 @@ DECODE_SOURCES = ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"]
 DECODE_SHA = "b36d81a54f38f0e6833eb54afe7b30de32d3c5f26ca7ac64b09690ae6d3fce86"
 PAIR_SOURCES = ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"]
 PAIR_SHA = "d334ae112e55900a4675c19d3a5e120f6ede0e0814cf43e52814b6296a4d8535"
-SPLIT_SOURCES = ["prefill_split.cuh", "common.cuh", "tc_ptx.cuh"]
-SPLIT_SHA = "ba5ade7553d65e90021c9814939ad7640c7124a3dc89340fefc6d13982c448df"
+PERSIST_SOURCES = ["prefill_persist.cuh", "common.cuh", "tc_ptx.cuh"]
+PERSIST_SHA = "e4210c033dc94d006173c98e097eeaf1013cd69caf0c0f5437b0eed06a12f2f6"
 CAPTURED_TRAFFIC = [
     {"workload": "decode_b8_n8000", "phase": "decode", "window": None, "hkv": None,
      "bytes": 267_997_440, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
@@ -182,13 +182,13 @@ CAPTURED_TRAFFIC = [
     {"workload": "swa_t32768", "phase": "decode", "window": None, "hkv": None,
      "bytes": 17_122_304, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": None, "hkv": None,
-     "bytes": 6_523_136, "sources": SPLIT_SOURCES, "sha256": SPLIT_SHA},
+     "bytes": 6_352_896, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": 256, "hkv": None,
      "bytes": 6_350_848, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": None,
      "bytes": 686_371_840, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": 32,
-     "bytes": 1_059_718_656, "sources": SPLIT_SOURCES, "sha256": SPLIT_SHA},
+     "bytes": 1_055_412_992, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
 ]
 
 
@@ -635,8 +635,9 @@ class PrefillStep:
 KERNEL_NAMES = {
     "simt": "prefill_simt_kernel (CUDA cores)",
     "pair": "pf2::prefill_pair_kernel (two query heads of one KV group per CTA)",
-    "split": "pfs::prefill_split_kernel (one query head per CTA; two softmax warpgroups over "
-           "keys 0-63 and 64-127 of each tile, each with its own running maximum, sum and O)",
+    "split": "pfp::prefill_persist_kernel (one query head per work item, one persistent CTA per "
+             "SM; two softmax warpgroups over keys 0-63 and 64-127 of each tile, each with its own "
+             "running maximum, sum and O; epilogue on its own warpgroup)",
 }
 
 

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "decode_splitk.cuh"
 #include "prefill_pair.cuh"
+#include "prefill_persist.cuh"
 #include "prefill_split.cuh"
 #include "simt.cuh"
 
@@ -383,6 +384,12 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
         !(prefill_prefers_split(B, Hq, Hkv, Tq, Tk, cached, seg != nullptr, window, di.sms)))
       return gqa::pf2::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached,
                               d, window, scale_log2, dev_status, st);
+    // One head per item: plain prompts on the persistent kernel (one CTA
+    // per SM walking its items), queries after a cache and packed segments
+    // on one CTA per item.
+    if (!cached && !seg)
+      return gqa::pfp::launch(q, k, v, o, seq_lens, B, Hq, Hkv, Tq, d, window, scale_log2,
+                              di.sms, dev_status, st);
     return gqa::pfs::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached, d,
                             window, scale_log2, dev_status, st);
   }

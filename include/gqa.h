@@ -330,9 +330,10 @@ int gqa_kv_head_for_query(int h, int Hq, int Hkv);
  * T cells, head width d and window (GQA_NO_WINDOW or w >= 1) on a device with
  * `sms` SMs:
  *   1  two query heads of one KV group per CTA (even group size), unless:
- *   2  one query head per CTA, its keys split over two softmax warpgroups
- *      (odd group size; or a prompt whose paired grid has fewer CTAs than
- *      `sms` and whose last query tile walks more than 4 KV tiles);
+ *   2  one query head per work item, its keys split over two softmax
+ *      warpgroups, on a persistent grid of one CTA per SM (odd group size;
+ *      or a prompt whose paired grid has fewer CTAs than `sms` and whose
+ *      last query tile walks more than 4 KV tiles);
  *   0  the CUDA-core kernel (d other than 64 or 128);
  *  -1  invalid arguments (non-positive sizes, Hq % Hkv != 0, bad window).
  * Host-only: reads nothing on the device and launches nothing. */

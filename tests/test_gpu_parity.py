@@ -91,6 +91,43 @@ def test_prefill_edge_cases(cuda_lib, case):
             assert torch.all(o[b, :, n:] == 0)
 
 
+LONG_ONE_HEAD = [
+    # (B, Hq, Hkv, T, d, window, lens): odd group sizes run one head per CTA;
+    # 65 query tiles per head orders the CTAs head by head
+    (2, 4, 4, 8229, 64, None, [8229, 6000]),
+    (1, 6, 2, 8229, 128, 1000, None),
+]
+
+
+@pytest.mark.parametrize("case", LONG_ONE_HEAD, ids=lambda c: f"B{c[0]}Hq{c[1]}Hkv{c[2]}T{c[3]}d{c[4]}w{c[5]}")
+def test_prefill_long_one_head_sampled_rows(cuda_lib, case):
+    """Long prompts on the one-head kernel in its head-by-head CTA order:
+    the first 256 rows of every head against the oracle's prefill, 48 seeded
+    random rows of every head against the oracle's row-by-row decode, and
+    rows past a sequence's length exact zeros."""
+    B, Hq, Hkv, T, d, window, lens = case
+    q, k, v = synthetic.qkv_prefill(B, Hq, Hkv, T, d, seed=300 + d, std=0.5)
+    lens_t = None if lens is None else torch.tensor(lens, dtype=torch.int32, device=DEV)
+    status = cuda_lib.new_status(DEV)
+    o = torch.full((B, Hq, T, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    cuda_lib.prefill(*_cuda(q, k, v), window=window, seq_lens=lens_t, out=o, status=status)
+    assert int(status.item()) == 0
+    T0 = 256
+    want = oracle.prefill(f64(q[:, :, :T0]), f64(k[:, :, :T0]), f64(v[:, :, :T0]), window=window)
+    assert_close(o[:, :, :T0], want, torch.bfloat16, f"first rows {case}")
+    n = lens or [T] * B
+    rng = np.random.default_rng(T)
+    cells = sorted(rng.choice(np.arange(T0, min(n)), size=48, replace=False).tolist())
+    k64, v64 = f64(k), f64(v)
+    got, want = [], []
+    for t in cells:
+        want.append(oracle.decode(f64(q[:, :, t]), k64, v64, [t + 1] * B, window=window))
+        got.append(f64(o[:, :, t]))
+    assert_close(np.stack(got), np.stack(want), torch.bfloat16, f"random rows {case}")
+    for b, nb in enumerate(n):
+        assert torch.all(o[b, :, nb:] == 0)
+
+
 def test_prefill_invalid_length_sets_status_and_zeroes(cuda_lib):
     q, k, v = _cuda(*synthetic.qkv_prefill(2, 4, 2, 64, 64, seed=5))
     status = cuda_lib.new_status(DEV)
