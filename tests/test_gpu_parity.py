@@ -138,6 +138,23 @@ def test_prefill_invalid_length_sets_status_and_zeroes(cuda_lib):
     assert torch.all(o[1] == 0)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (6, 2)], ids=["mha", "group3"])
+def test_prefill_one_head_invalid_and_empty_lengths(cuda_lib, Hq, Hkv):
+    """The persistent one-head kernel: a sequence with an invalid length is
+    written as zeros and reported, an empty one as zeros, the others exact."""
+    B, T, d = 3, 300, 64
+    q, k, v = synthetic.qkv_prefill(B, Hq, Hkv, T, d, seed=9)
+    lens = [T, T + 1, 0]
+    status = cuda_lib.new_status(DEV)
+    o = torch.full((B, Hq, T, d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    cuda_lib.prefill(*_cuda(q, k, v), seq_lens=torch.tensor(lens, dtype=torch.int32, device=DEV),
+                     out=o, status=status)
+    assert int(status.item()) == 5
+    want = oracle.prefill(f64(q[:1]), f64(k[:1]), f64(v[:1]))
+    assert_close(o[:1], want, torch.bfloat16, "valid sequence")
+    assert torch.all(o[1:] == 0)
+
+
 def test_prefill_empty(cuda_lib):
     q = torch.empty((0, 4, 8, 64), dtype=torch.bfloat16, device=DEV)
     k = torch.empty((0, 2, 8, 64), dtype=torch.bfloat16, device=DEV)
