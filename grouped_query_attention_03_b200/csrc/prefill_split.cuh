@@ -8,9 +8,10 @@
 // max/sum from "GQA, FlashAttention and the KV cache"): for every batch row
 // b, query head h and active cell t < n_b, softmax over the permitted keys
 // of scale * q.k, mixed with the value rows of the shared lane g(h);
-// inactive rows are zero.  It serves odd group sizes (MHA included), which
-// the paired kernel (prefill_pair.cuh) cannot, and short prompts whose
-// paired grid would leave SMs idle.
+// inactive rows are zero.  It serves queries after a cache (the multi-token
+// decode) and packed prompts of odd group sizes (MHA included), which the
+// paired kernel (prefill_pair.cuh) cannot; plain prompts of those shapes run
+// the same arithmetic on the persistent kernel (prefill_persist.cuh).
 //
 // One CTA owns a 128-row query tile of one (b, h) and walks the 128-key
 // tiles that intersect its permitted band, skipping tiles wholly outside
