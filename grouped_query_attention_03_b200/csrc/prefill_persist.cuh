@@ -64,7 +64,10 @@ struct Cfg {
   static constexpr int KB = D / 64;                 // 64-column blocks
   static constexpr int BLK = kBM * 128;             // 128 rows x 128 B = 16 KB
   static constexpr int TILE = KB * BLK;             // a Q, K or V tile
+  // K/V stages; equal to the number of S buffers, so that S[s] complete
+  // also means K stage s is free and P V[s] complete that V stage s is.
   static constexpr int STAGES = 2;
+  static_assert(STAGES == 2, "S buffers and K/V stages share their index");
   static constexpr int NQ = 2;                      // Q buffers
   static constexpr int NOB = (D == 64) ? 2 : 1;     // O buffers in TMEM
   static constexpr int OFF_Q = 0;
@@ -90,10 +93,12 @@ struct Params {
 
 struct Bars {
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
-  uint64_t s_full[2];     // S[s] written by the MMA
+  uint64_t k_full[2], v_full[2];
+  // S[s] written by the MMA; also K stage s read (the stage and the S
+  // buffer of a KV tile have the same index, so no separate commit)
+  uint64_t s_full[2];
   uint64_t p_full[2][2];  // [s][half]: that half's P written over S[s]
-  uint64_t pv_done[2];    // both halves' P V of an S[s] tile complete
+  uint64_t pv_done[2];    // both halves' P V of an S[s] tile complete; V stage s read
   uint64_t o_done[2];     // an item's last P V into O buffer [ob] complete
   uint64_t o_free[2];     // the epilogue has read O buffer [ob]
   uint64_t ml_full[2];    // both halves' (maximum, sum) of the item in [ob] posted
@@ -172,8 +177,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars.q_empty[s], 1);
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.k_empty[s], 1);
-      mbar_init(&bars.v_empty[s], 1);
       mbar_init(&bars.s_full[s], 1);
       mbar_init(&bars.p_full[s][0], 4);  // the half's four warps
       mbar_init(&bars.p_full[s][1], 4);
@@ -448,14 +451,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < x.nt; ++j) {
             const int tg = tcg + j, s = tg % K::STAGES;
             const int krow = (x.j0 + j) * kBN;
-            if (tg >= K::STAGES && !mbar_wait(&bars.k_empty[s], ((tg / K::STAGES) - 1) & 1, &failed)) break;
+            // stage s is free once S of the tile two back is complete
+            if (tg >= K::STAGES && !mbar_wait(&bars.s_full[s], ((tg / K::STAGES) - 1) & 1, &failed)) break;
             mbar_arrive_expect_tx(&bars.k_full[s], K::TILE);
 #pragma unroll
             for (int cc = 0; cc < K::KB; ++cc)
               tc::tma_load_3d(smem + K::OFF_K + s * K::TILE + cc * K::BLK, &tmK, cc * 64, krow,
                               x.b * p.Hkv + x.g, &bars.k_full[s]);
             kf[s]++;
-            if (tg >= K::STAGES && !mbar_wait(&bars.v_empty[s], ((tg / K::STAGES) - 1) & 1, &failed)) break;
+            if (tg >= K::STAGES && !mbar_wait(&bars.pv_done[s], ((tg / K::STAGES) - 1) & 1, &failed)) break;
             mbar_arrive_expect_tx(&bars.v_full[s], K::TILE);
 #pragma unroll
             for (int cc = 0; cc < K::KB; ++cc)
@@ -513,7 +517,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             tc::mma_commit(&bars.pv_done[s]);
-            tc::mma_commit(&bars.v_empty[vs]);
             return true;
           };
           if (!mbar_wait(&bars.q_full[qb], (ai / K::NQ) & 1, &failed)) break;
@@ -533,7 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             issued = true;
             tc::mma_commit(&bars.s_full[sb]);
-            tc::mma_commit(&bars.k_empty[ks]);
             if (j == x.nt - 1) tc::mma_commit(&bars.q_empty[qb]);  // Q read by its last S
             if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
           }
