@@ -46,8 +46,10 @@
 // workspace needs no clearing between calls.  No CTA ever waits for another.
 //
 // Launched as a programmatic dependent of the previous kernel on the stream:
-// a CTA sets up its barriers while that kernel drains, then waits for it to
-// complete (griddepcontrol.wait) before its first access to global memory.
+// a CTA sets up its barriers and asks L2 for the first cache rows of its
+// range (planned from the lengths as they read then) while that kernel
+// drains, then waits for it to complete (griddepcontrol.wait) before it
+// reads anything it uses or writes anything.
 #pragma once
 
 #include <cuda.h>
@@ -188,6 +190,116 @@ __device__ __forceinline__ int extent(const Params &p, int len) {
 // swizzled box (the TMA swizzle XORs the chunk index with r mod 8).
 __device__ __forceinline__ int swz(int r, int ch) {
   return r * 128 + ((ch ^ (r & 7)) << 4);
+}
+
+// ---------------------------------------------------- prefetch before wait
+// Rows of its range a CTA asks L2 for before the previous kernel on the
+// stream has completed (a cap, so that the prefetched rows of every CTA fit
+// in L2 together with room to spare: 148 CTAs x 512 rows x 512 B at d = 128
+// is 39 MB of the 126 MB).
+constexpr int kPrefetchRows = 512;
+
+// Runs on the producer warp before griddepcontrol.wait, while the previous
+// kernel drains: plans this CTA's range as the producer will (same row
+// space, same split) from the lengths as they read now, and asks L2 for
+// the first kPrefetchRows cache rows of it (K and V, whole TMA boxes).  The
+// lengths may be stale -- a fused append of the previous step may still be
+// advancing them -- so this is only a hint: it writes nothing but the
+// shared length cache (which the producer fills again after the wait), and
+// the producer plans again from the lengths it reads then.  The lengths
+// are read through L2 only (ld.global.cg), so no line of them sits in this
+// SM's L1 when the producer reads them after the wait.  Invalid lengths,
+// or more sequences than the shared cache holds, prefetch nothing.
+template <int D, int R>
+__device__ void prefetch_range(const Params &p, const CUtensorMap *tmK,
+                               const CUtensorMap *tmV, int *s_len) {
+  using K = Cfg<D, R>;
+  const int lane = threadIdx.x & 31;
+  const int G = gridDim.x, c = blockIdx.x;
+  if (!p.lens_smem) return;
+  long long tot = 0;
+  int bad_local = 0;
+  for (int b = lane; b < p.B; b += 32) {
+    const int n = __ldcg(p.seq_lens + b) + p.add;
+    s_len[b] = n;
+    bad_local |= (n < p.add || (!p.ring && n > p.C));
+    tot += extent(p, eligible_cells(p, max(n, 0)));
+  }
+  if (__any_sync(0xffffffffu, bad_local)) return;
+  __syncwarp();
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, off);
+  const long long total = tot * p.VL;
+  long long per = udiv(total + G - 1, G);
+  if (per < p.min_rows) per = p.min_rows;
+  const long long start = (long long)c * per;
+  const long long end = min(min(total, start + per), start + kPrefetchRows);
+  if (start >= end) return;
+  // the batch row holding row `start` (warp prefix scan, as the producer)
+  long long cum = 0, cum_b = 0;
+  int b = -1;
+  for (int b0 = 0; b0 < p.B && b < 0; b0 += 32) {
+    const int bb = b0 + lane;
+    const long long x = bb < p.B ? (long long)extent(p, eligible_cells(p, s_len[bb])) * p.VL : 0;
+    long long incl = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, cum + incl > start);
+    if (hit) {
+      const int src = __ffs(hit) - 1;
+      b = b0 + src;
+      cum_b = cum + __shfl_sync(0xffffffffu, incl - x, src);
+    } else {
+      cum += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  if (b < 0) return;
+  int n_b = s_len[b];
+  int len = eligible_cells(p, n_b);
+  int ext = extent(p, len);
+  int lo = first_cell(p, n_b, len);
+  const long long off0 = start - cum_b;
+  int vl = (int)udiv(off0, ext);
+  int row = (int)(off0 - (long long)vl * ext) - p.pad;
+  long long pos = start;
+  while (pos < end) {
+    if (row < 0) {  // the lane's virtual rows
+      pos -= row;
+      row = 0;
+      if (pos >= end) break;
+    }
+    const int nrows = (int)min((long long)(len - row), end - pos);
+    const int y0 = (b * p.Hkv + vl / p.nsub) * p.C + lo + row;
+    const int nbox = (nrows + K::ROWS - 1) / K::ROWS;
+    for (int i = lane; i < nbox; i += 32) {
+#pragma unroll
+      for (int kb = 0; kb < K::KB; ++kb) {
+        tc::tma_prefetch_2d(tmK, kb * 64, y0 + i * K::ROWS);
+        tc::tma_prefetch_2d(tmV, kb * 64, y0 + i * K::ROWS);
+      }
+    }
+    pos += nrows;
+    row = -p.pad;
+    if (++vl == p.VL) {
+      vl = 0;
+      // next batch row with cells to read (warp-parallel search)
+      int nb = -1;
+      for (int b0 = b + 1; b0 < p.B && nb < 0; b0 += 32) {
+        const int bb = b0 + lane;
+        const unsigned m = __ballot_sync(0xffffffffu, bb < p.B && eligible_cells(p, s_len[bb]) > 0);
+        if (m) nb = b0 + __ffs(m) - 1;
+      }
+      if (nb < 0) return;
+      b = nb;
+      n_b = s_len[b];
+      len = eligible_cells(p, n_b);
+      ext = extent(p, len);
+      lo = first_cell(p, n_b, len);
+    }
+  }
 }
 
 // -------------------------------------------------------------- producer
@@ -820,10 +932,13 @@ __global__ void __launch_bounds__(Cfg<D, R>::THREADS, Cfg<D, R>::MIN_BLOCKS)
   }
   __syncthreads();
   // Everything above touches only shared memory and the kernel parameters.
-  // From here on the CTA reads and writes global memory that the previous
+  // The producer warp then asks L2 for the first rows of this CTA's range
+  // (reads only, planned from lengths that may still change).  From the
+  // wait on, the CTA reads and writes global memory that the previous
   // kernel on the stream may use: wait until it has completed (a no-op when
   // the launch is not a programmatic dependent), then let the next kernel
   // start its own set-up.
+  if (warp == K::NWC) prefetch_range<D, R>(p, &tmK, &tmV, s_len);
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
   if (warp == K::NWC) {

@@ -226,6 +226,16 @@ __device__ __forceinline__ void st_global_hint(float2 *addr, float2 v, uint64_t 
 }
 
 // tma_load_2d with an L2 cache policy.
+// Ask L2 for one tile of a 2D tensor map (its box at {c0, c1}); nothing is
+// written to shared memory and no barrier is signalled.  c0 * element size
+// must be a multiple of 16 bytes; rows outside the tensor fetch nothing.
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_hint(void *smem_dst, const CUtensorMap *map,
                                                  int c0, int c1, uint64_t *bar,
                                                  uint64_t policy) {
