@@ -167,28 +167,28 @@ def pass_stats(ms):
 # lines stripped: once the code changes the figure no longer describes the
 # kernel and is reported as null (a comment edit does not count).
 DECODE_SOURCES = ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"]
-DECODE_SHA = "b36d81a54f38f0e6833eb54afe7b30de32d3c5f26ca7ac64b09690ae6d3fce86"
+DECODE_SHA = "9fa112902e5b540a87fab647558588cf17164bbb3744533a4eea05ebbd374f75"
 PAIR_SOURCES = ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"]
-PAIR_SHA = "d334ae112e55900a4675c19d3a5e120f6ede0e0814cf43e52814b6296a4d8535"
+PAIR_SHA = "2407996e7ea83134b91dadf5de67932570acb9f83027ac970d43d980b81517d3"
 PERSIST_SOURCES = ["prefill_persist.cuh", "common.cuh", "tc_ptx.cuh"]
-PERSIST_SHA = "e4210c033dc94d006173c98e097eeaf1013cd69caf0c0f5437b0eed06a12f2f6"
+PERSIST_SHA = "65704b8aa2799423ea8e9ef25fab9a4c754ccff8dc9972f0e401f72b8c000bba"
 CAPTURED_TRAFFIC = [
     {"workload": "decode_b8_n8000", "phase": "decode", "window": None, "hkv": None,
-     "bytes": 267_997_440, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 268_544_768, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "decode_ragged", "phase": "decode", "window": None, "hkv": 1,
-     "bytes": 148_572_928, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 148_251_392, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "decode_ragged", "phase": "decode", "window": None, "hkv": 8,
-     "bytes": 1_124_909_120, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 1_125_872_296, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "swa_t32768", "phase": "decode", "window": None, "hkv": None,
-     "bytes": 17_122_304, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 17_116_928, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": None, "hkv": None,
      "bytes": 6_352_896, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": 256, "hkv": None,
-     "bytes": 6_350_848, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 6_355_200, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": None,
-     "bytes": 686_371_840, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 685_640_704, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": 32,
-     "bytes": 1_055_412_992, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
+     "bytes": 1_060_582_144, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
 ]
 
 
