@@ -302,6 +302,15 @@ __device__ void prefetch_range(const Params &p, const CUtensorMap *tmK,
   }
 }
 
+// Transpose of an 8x8 bf16 tile held as an MMA fragment (thread (g, t) has
+// row g, columns 2t and 2t+1 packed): afterwards thread (g, t) has row g of
+// the transpose, i.e. rows 2t and 2t+1 of column g.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // -------------------------------------------------------------- producer
 template <int D, int R>
 __device__ void producer(const Params &p, const CUtensorMap *tmK,
@@ -622,9 +631,15 @@ __device__ void consumer(const Params &p, unsigned char *smem,
   const int g = lane >> 2, t = lane & 3;
   bool failed = false;
 
-  uint32_t qa[KS][4];      // Q tile, A operand, per 16-feature k-step
-  float o[NT][4];          // O tile accumulators
-  float m_run[2], l_run[2];  // head rows g and g + 8
+  // Up to 8 heads (TR) the products are taken transposed, S^T = K Q^T and
+  // O^T += V^T P^T: a warp's 16 cache rows fill the MMA's 16-row dimension
+  // and the heads its 8 columns, 8 + 8 MMAs per 16 cache rows where the
+  // heads as tile rows (up to 16) take 16 + 16.
+  constexpr bool TR = R <= 8;
+  constexpr int NO = TR ? D / 16 : NT;
+  uint32_t qa[KS][TR ? 2 : 4];  // Q per 16-feature k-step: B operand (TR), else A
+  float o[NO][4];               // O^T tiles of 16 features (TR), else O tiles of 8
+  float m_run[2], l_run[2];     // TR: head columns 2t, 2t + 1; else head rows g, g + 8
   int stage_count = 0, comb_count = 0;
   // Split lanes whose partial this CTA wrote, counted at the end (at most
   // two: the first and the last segment of the range).
@@ -650,13 +665,18 @@ __device__ void consumer(const Params &p, unsigned char *smem,
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         const int c0 = ks * 16 + 2 * t;
-        qa[ks][0] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0) : 0u;
-        qa[ks][1] = g + 8 < rc ? *reinterpret_cast<const uint32_t *>(sQ + (g + 8) * D + c0) : 0u;
-        qa[ks][2] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0 + 8) : 0u;
-        qa[ks][3] = g + 8 < rc ? *reinterpret_cast<const uint32_t *>(sQ + (g + 8) * D + c0 + 8) : 0u;
+        if constexpr (TR) {  // B[k][n] = Q[n][k]: features 2t, 2t+1 (+8) of head g
+          qa[ks][0] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0) : 0u;
+          qa[ks][1] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0 + 8) : 0u;
+        } else {
+          qa[ks][0] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0) : 0u;
+          qa[ks][1] = g + 8 < rc ? *reinterpret_cast<const uint32_t *>(sQ + (g + 8) * D + c0) : 0u;
+          qa[ks][2] = g < rc ? *reinterpret_cast<const uint32_t *>(sQ + g * D + c0 + 8) : 0u;
+          qa[ks][3] = g + 8 < rc ? *reinterpret_cast<const uint32_t *>(sQ + (g + 8) * D + c0 + 8) : 0u;
+        }
       }
 #pragma unroll
-      for (int n = 0; n < NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+      for (int n = 0; n < NO; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
       m_run[0] = m_run[1] = -INFINITY;
       l_run[0] = l_run[1] = 0.f;
     }
@@ -697,83 +717,154 @@ __device__ void consumer(const Params &p, unsigned char *smem,
       __syncwarp();
     }
 
-    if (nv > 0) {
-      // ---- S = Q K^T for this warp's 16 cache rows (two 8-row tiles)
-      float s[2][4];
+    if constexpr (TR) {
+      if (nv > 0) {
+        // ---- S^T = K Q^T: the warp's 16 cache rows x 8 head columns (two
+        // accumulators over alternate k-steps, so the chains are half as long)
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+        const int krow = w * kBR + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-        const int krow = w * kBR + nt * 8 + (lane & 7);
-#pragma unroll
-        for (int kk = 0; kk < KS / 2; ++kk) {
-          const int ch = 4 * kk + (lane >> 3);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(sK + (ch >> 3) * K::BOX + swz(krow, ch & 7), b0, b1, b2, b3);
-          mma_16816(s[nt], qa[2 * kk], b0, b1);
-          mma_16816(s[nt], qa[2 * kk + 1], b2, b3);
+        for (int ks = 0; ks < KS; ++ks) {
+          const int ch = 2 * ks + (lane >> 4);
+          uint32_t a[4];
+          ldsm_x4(sK + (ch >> 3) * K::BOX + swz(krow, ch & 7), a[0], a[1], a[2], a[3]);
+          mma_16816((ks & 1) ? s2 : s, a, qa[ks][0], qa[ks][1]);
         }
-      }
-      // ---- online softmax on the fragments (log2 domain)
-      float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        // ---- online softmax over the rows (log2 domain): this thread has
+        // rows g and g + 8 of head columns 2t and 2t + 1
+        const bool r0 = g < nv, r1 = g + 8 < nv;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int col = nt * 8 + 2 * t + (e & 1);
-          const float v = col < nv ? s[nt][e] * p.scale_log2 : -INFINITY;
-          s[nt][e] = v;
-          mx[e >> 1] = fmaxf(mx[e >> 1], v);
+          const float v = s[e] + s2[e];
+          s[e] = (e < 2 ? r0 : r1) ? v * p.scale_log2 : -INFINITY;
         }
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
-        mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
-        if (mx[i] > m_run[i] + kLazyRescale) {
-          const float alpha = exp2f(m_run[i] - mx[i]);  // 0 when m_run = -inf
-          l_run[i] *= alpha;
-          m_run[i] = mx[i];
+        for (int j = 0; j < 2; ++j) {
+          float mx = fmaxf(s[j], s[j + 2]);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          if (mx > m_run[j] + kLazyRescale) {
+            const float alpha = exp2f(m_run[j] - mx);  // 0 when m_run = -inf
+            l_run[j] *= alpha;
+            m_run[j] = mx;
 #pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            o[n][2 * i] *= alpha;
-            o[n][2 * i + 1] *= alpha;
+            for (int n = 0; n < NO; ++n) {
+              o[n][j] *= alpha;
+              o[n][j + 2] *= alpha;
+            }
           }
         }
-      }
-      uint32_t pa[4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
         float pv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float msub = m_run[e >> 1] == -INFINITY ? 0.f : m_run[e >> 1];
-          pv[e] = exp2f(s[nt][e] - msub);
+          const float msub = m_run[e & 1] == -INFINITY ? 0.f : m_run[e & 1];
+          pv[e] = exp2f(s[e] - msub);
         }
-        pa[2 * nt] = pack_bf16(pv[0], pv[1]);
-        pa[2 * nt + 1] = pack_bf16(pv[2], pv[3]);
+        const uint32_t p0 = pack_bf16(pv[0], pv[1]);  // row g: heads 2t, 2t + 1
+        const uint32_t p1 = pack_bf16(pv[2], pv[3]);  // row g + 8
         // the denominator sums exactly the bf16 weights the MMA uses
-        l_run[0] += bf16lo_to_f32(pa[2 * nt]) + bf16hi_to_f32(pa[2 * nt]);
-        l_run[1] += bf16lo_to_f32(pa[2 * nt + 1]) + bf16hi_to_f32(pa[2 * nt + 1]);
-      }
-      // ---- O += P V (A = P over the 16 cache rows, B = V rows from smem)
-      const int vrow = w * kBR + (lane & 7) + ((lane >> 3) & 1) * 8;
+        l_run[0] += bf16lo_to_f32(p0) + bf16lo_to_f32(p1);
+        l_run[1] += bf16hi_to_f32(p0) + bf16hi_to_f32(p1);
+        // P^T as the B operand: rows 2t, 2t + 1 (and + 8) of head column g
+        const uint32_t pb0 = movmatrix_t(p0), pb1 = movmatrix_t(p1);
+        // ---- O^T += V^T P^T (A = V^T by transposing loads, 16 features a tile)
+        const int vrow = w * kBR + (lane & 7) + ((lane >> 4) & 1) * 8;
 #pragma unroll
-      for (int nn = 0; nn < NT / 2; ++nn) {
-        const int ch = 2 * nn + (lane >> 4);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sV + (ch >> 3) * K::BOX + swz(vrow, ch & 7), b0, b1, b2, b3);
-        mma_16816(o[2 * nn], pa, b0, b1);
-        mma_16816(o[2 * nn + 1], pa, b2, b3);
+        for (int n = 0; n < NO; ++n) {
+          const int ch = 2 * n + ((lane >> 3) & 1);
+          uint32_t a[4];
+          ldsm_x4_t(sV + (ch >> 3) * K::BOX + swz(vrow, ch & 7), a[0], a[1], a[2], a[3]);
+          mma_16816(o[n], a, pb0, pb1);
+        }
+      }
+    } else {
+      if (nv > 0) {
+        // ---- S = Q K^T for this warp's 16 cache rows (two 8-row tiles)
+        float s[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+          const int krow = w * kBR + nt * 8 + (lane & 7);
+#pragma unroll
+          for (int kk = 0; kk < KS / 2; ++kk) {
+            const int ch = 4 * kk + (lane >> 3);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(sK + (ch >> 3) * K::BOX + swz(krow, ch & 7), b0, b1, b2, b3);
+            mma_16816(s[nt], qa[2 * kk], b0, b1);
+            mma_16816(s[nt], qa[2 * kk + 1], b2, b3);
+          }
+        }
+        // ---- online softmax on the fragments (log2 domain)
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = nt * 8 + 2 * t + (e & 1);
+            const float v = col < nv ? s[nt][e] * p.scale_log2 : -INFINITY;
+            s[nt][e] = v;
+            mx[e >> 1] = fmaxf(mx[e >> 1], v);
+          }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 1));
+          mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], 2));
+          if (mx[i] > m_run[i] + kLazyRescale) {
+            const float alpha = exp2f(m_run[i] - mx[i]);  // 0 when m_run = -inf
+            l_run[i] *= alpha;
+            m_run[i] = mx[i];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+              o[n][2 * i] *= alpha;
+              o[n][2 * i + 1] *= alpha;
+            }
+          }
+        }
+        uint32_t pa[4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          float pv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float msub = m_run[e >> 1] == -INFINITY ? 0.f : m_run[e >> 1];
+            pv[e] = exp2f(s[nt][e] - msub);
+          }
+          pa[2 * nt] = pack_bf16(pv[0], pv[1]);
+          pa[2 * nt + 1] = pack_bf16(pv[2], pv[3]);
+          // the denominator sums exactly the bf16 weights the MMA uses
+          l_run[0] += bf16lo_to_f32(pa[2 * nt]) + bf16hi_to_f32(pa[2 * nt]);
+          l_run[1] += bf16lo_to_f32(pa[2 * nt + 1]) + bf16hi_to_f32(pa[2 * nt + 1]);
+        }
+        // ---- O += P V (A = P over the 16 cache rows, B = V rows from smem)
+        const int vrow = w * kBR + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int nn = 0; nn < NT / 2; ++nn) {
+          const int ch = 2 * nn + (lane >> 4);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(sV + (ch >> 3) * K::BOX + swz(vrow, ch & 7), b0, b1, b2, b3);
+          mma_16816(o[2 * nn], pa, b0, b1);
+          mma_16816(o[2 * nn + 1], pa, b2, b3);
+        }
       }
     }
 
     // ---- end of a lane segment: combine the warps, then output or partial
     if (hd.flags & kLast) {
+      // the sums over the warp's rows: the four lanes sharing a head row, or
+      // (TR) the eight sharing a head column
       float l_tot[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         float l = l_run[i];
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if constexpr (TR) {
+          l += __shfl_xor_sync(0xffffffffu, l, 4);
+          l += __shfl_xor_sync(0xffffffffu, l, 8);
+          l += __shfl_xor_sync(0xffffffffu, l, 16);
+        } else {
+          l += __shfl_xor_sync(0xffffffffu, l, 1);
+          l += __shfl_xor_sync(0xffffffffu, l, 2);
+        }
         l_tot[i] = l;
       }
       // Every warp is done with this stage: reuse it as scratch.
@@ -781,20 +872,40 @@ __device__ void consumer(const Params &p, unsigned char *smem,
       float *sm_m = reinterpret_cast<float *>(base);   // [NWC][16]
       float *sm_l = sm_m + NWC * 16;                     // [NWC][16]
       float *sm_acc = sm_l + NWC * 16;                   // [NWC][R][ACC_STRIDE]
-      if (t == 0) {
-        sm_m[w * 16 + g] = m_run[0];
-        sm_l[w * 16 + g] = l_tot[0];
-        sm_m[w * 16 + g + 8] = m_run[1];
-        sm_l[w * 16 + g + 8] = l_tot[1];
-      }
+      if constexpr (TR) {
+        // O^T tile n: features 16n + g (+ 8) of head columns 2t, 2t + 1
+        if (g == 0) {
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        if (g < R)
-          *reinterpret_cast<float2 *>(sm_acc + (w * R + g) * K::ACC_STRIDE + n * 8 + 2 * t) =
-              make_float2(o[n][0], o[n][1]);
-        if (g + 8 < R)
-          *reinterpret_cast<float2 *>(sm_acc + (w * R + g + 8) * K::ACC_STRIDE + n * 8 + 2 * t) =
-              make_float2(o[n][2], o[n][3]);
+          for (int j = 0; j < 2; ++j) {
+            sm_m[w * 16 + 2 * t + j] = m_run[j];
+            sm_l[w * 16 + 2 * t + j] = l_tot[j];
+          }
+        }
+#pragma unroll
+        for (int n = 0; n < NO; ++n)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (2 * t + j < R) {
+              float *row = sm_acc + (w * R + 2 * t + j) * K::ACC_STRIDE + n * 16 + g;
+              row[0] = o[n][j];
+              row[8] = o[n][j + 2];
+            }
+      } else {
+        if (t == 0) {
+          sm_m[w * 16 + g] = m_run[0];
+          sm_l[w * 16 + g] = l_tot[0];
+          sm_m[w * 16 + g + 8] = m_run[1];
+          sm_l[w * 16 + g + 8] = l_tot[1];
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          if (g < R)
+            *reinterpret_cast<float2 *>(sm_acc + (w * R + g) * K::ACC_STRIDE + n * 8 + 2 * t) =
+                make_float2(o[n][0], o[n][1]);
+          if (g + 8 < R)
+            *reinterpret_cast<float2 *>(sm_acc + (w * R + g + 8) * K::ACC_STRIDE + n * 8 + 2 * t) =
+                make_float2(o[n][2], o[n][3]);
+        }
       }
       csync(comb, comb_count, &failed);
       const int L = hd.lane, b = L / p.VL, vl = L % p.VL;
