@@ -167,28 +167,28 @@ def pass_stats(ms):
 # lines stripped: once the code changes the figure no longer describes the
 # kernel and is reported as null (a comment edit does not count).
 DECODE_SOURCES = ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"]
-DECODE_SHA = "9fa112902e5b540a87fab647558588cf17164bbb3744533a4eea05ebbd374f75"
+DECODE_SHA = "f5815f28d2eec9e95b0d4534fc3a003f3b7bcf1c684160196fa61561e521d95b"
 PAIR_SOURCES = ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"]
-PAIR_SHA = "2407996e7ea83134b91dadf5de67932570acb9f83027ac970d43d980b81517d3"
+PAIR_SHA = "ccbbdc5d3860c03427642dfeab5c45eab3e4763a1b456fb20d8a743e2a3ace59"
 PERSIST_SOURCES = ["prefill_persist.cuh", "common.cuh", "tc_ptx.cuh"]
-PERSIST_SHA = "65704b8aa2799423ea8e9ef25fab9a4c754ccff8dc9972f0e401f72b8c000bba"
+PERSIST_SHA = "18ab7f655a08bbee094ebf3a12788f9f826b987aaea6f4c00b9eff2a8c749338"
 CAPTURED_TRAFFIC = [
     {"workload": "decode_b8_n8000", "phase": "decode", "window": None, "hkv": None,
-     "bytes": 268_544_768, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 268_040_448, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "decode_ragged", "phase": "decode", "window": None, "hkv": 1,
-     "bytes": 148_251_392, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 148_212_992, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "decode_ragged", "phase": "decode", "window": None, "hkv": 8,
-     "bytes": 1_125_872_296, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 1_125_684_880, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "swa_t32768", "phase": "decode", "window": None, "hkv": None,
-     "bytes": 17_116_928, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
+     "bytes": 17_117_952, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": None, "hkv": None,
-     "bytes": 6_352_896, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
+     "bytes": 6_356_736, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": 256, "hkv": None,
-     "bytes": 6_355_200, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 6_352_896, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": None,
-     "bytes": 685_640_704, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 699_909_888, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": 32,
-     "bytes": 1_060_582_144, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
+     "bytes": 1_055_563_264, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
 ]
 
 

@@ -383,7 +383,7 @@ gqa_status attend_impl(gqa_dtype dtype, const void *q, const void *k,
     if (gqa::pf2::supported(d, Hq, Hkv) &&
         !(prefill_prefers_split(B, Hq, Hkv, Tq, Tk, cached, seg != nullptr, window, di.sms)))
       return gqa::pf2::launch(q, k, v, o, seq_lens, seg, B, Hq, Hkv, Tq, Tk, cached,
-                              d, window, scale_log2, dev_status, st);
+                              d, window, scale_log2, di.sms, dev_status, st);
     // One head per item: plain prompts on the persistent kernel (one CTA
     // per SM walking its items), queries after a cache and packed segments
     // on one CTA per item.

@@ -58,6 +58,10 @@ constexpr int kRegsLow = 72, kRegsHigh = 216;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxSlots = 12;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// K/V tiles a CTA of a one-wave grid asks L2 for before the dependency
+// wait, with its two Q tiles (148 CTAs x 6 tiles x 32 KB at d = 128 is
+// 28 MB).
+constexpr int kPrefetchTiles = 4;
 
 template <int D>
 struct Cfg {
@@ -86,6 +90,8 @@ struct Params {
   const int32_t *seg;  // prompt only: [B,Tq] first key cell of row t's
                        // packed segment, or NULL (segment start 0)
   float scale_log2;
+  int prefetch;  // 1: the grid fits in one wave; its tiles are asked of L2
+                 // before the dependency wait
 };
 
 // First permitted key of query position t ("Intersect the window with the
@@ -308,9 +314,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  // Barriers and TMEM are set up; from here on the CTA reads memory the
-  // previous kernel on the stream may write: wait for it (a no-op unless
-  // launched as a programmatic dependent), then let the next one start.
+  // Barriers and TMEM are set up.  While the previous kernel on the stream
+  // drains, the producer of a grid that fits in one wave asks L2 for both
+  // Q tiles and the first K/V tiles of a plain prompt's tile (reads only,
+  // planned as if the sequence had all Tk rows: no length is read before
+  // the wait; later waves start after the previous kernel anyway).  From
+  // the wait on, the CTA reads memory the previous kernel may write: wait
+  // for it (a no-op unless launched as a programmatic dependent), then let
+  // the next one start.
+  if (!SEG && p.prefetch && !p.cached && warp == 0 && lane == 0) {
+    const int lo0 = p.window > 0 ? max(0, m0 - (p.window - 1)) : 0;
+    const int hi0 = min(m0 + kBM - 1, p.Tk - 1);
+    const int jf = lo0 / kBN, nf = m0 < p.Tk ? min(hi0 / kBN - jf + 1, kPrefetchTiles) : 0;
+#pragma unroll
+    for (int cc = 0; cc < K::KB; ++cc) {
+      if (nf > 0) {
+        tc::tma_prefetch_3d(&tmQ, cc * 64, m0, b * p.Hq + h0);
+        tc::tma_prefetch_3d(&tmQ, cc * 64, m0, b * p.Hq + h0 + 1);
+      }
+      for (int j = 0; j < nf; ++j) {
+        tc::tma_prefetch_3d(&tmK, cc * 64, (jf + j) * kBN, b * p.Hkv + g);
+        tc::tma_prefetch_3d(&tmV, cc * 64, (jf + j) * kBN, b * p.Hkv + g);
+      }
+    }
+  }
   griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
   // n_b keys of sequence b; `rows` query rows produce output, the query
@@ -523,7 +550,7 @@ template <int D>
 gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
                     const int32_t *lens, const int32_t *seg, int B, int Hq, int Hkv,
                     int Tq, int Tk, int cached, int window, float scale_log2,
-                    int32_t *status, cudaStream_t st) {
+                    int sms, int32_t *status, cudaStream_t st) {
   using K = Cfg<D>;
   CUtensorMap mq, mk, mv;
   if (!tma::make_bf16_map(&mq, q, D, Tq, B * Hq, 128) ||
@@ -560,6 +587,7 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
   p.scale_log2 = scale_log2;
   const long long grid = (long long)B * Hkv * p.pairs * p.num_mt;
   if (grid > 0x7fffffffLL) return GQA_ERR_UNSUPPORTED;
+  p.prefetch = grid <= sms ? 1 : 0;
   const cudaError_t e =
       seg ? launch_dependent(prefill_pair_kernel<D, true>, dim3((unsigned)grid), dim3(kThreads),
                              K::SMEM, st, mq, mk, mv, p)
@@ -577,12 +605,12 @@ gqa_status launch_d(const void *q, const void *k, const void *v, void *o,
 inline gqa_status launch(const void *q, const void *k, const void *v, void *o,
                          const int32_t *lens, const int32_t *seg, int B, int Hq, int Hkv,
                          int Tq, int Tk, int cached, int d, int window, float scale_log2,
-                         int32_t *status, cudaStream_t st) {
+                         int sms, int32_t *status, cudaStream_t st) {
   if (d == 64)
     return launch_d<64>(q, k, v, o, lens, seg, B, Hq, Hkv, Tq, Tk, cached, window,
-                        scale_log2, status, st);
+                        scale_log2, sms, status, st);
   return launch_d<128>(q, k, v, o, lens, seg, B, Hq, Hkv, Tq, Tk, cached, window,
-                       scale_log2, status, st);
+                       scale_log2, sms, status, st);
 }
 
 }  // namespace pf2

@@ -226,6 +226,15 @@ __device__ __forceinline__ void st_global_hint(float2 *addr, float2 v, uint64_t 
 }
 
 // tma_load_2d with an L2 cache policy.
+// Ask L2 for one box of a 3D tensor map at {c0, c1, c2}; the same rules as
+// tma_prefetch_2d below.
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
 // Ask L2 for one tile of a 2D tensor map (its box at {c0, c1}); nothing is
 // written to shared memory and no barrier is signalled.  c0 * element size
 // must be a multiple of 16 bytes; rows outside the tensor fetch nothing.
