@@ -71,6 +71,8 @@ FUSED_CASES = [
     (4100, 2, 1, 4, 128, [b % 4 for b in range(4100)], None),  # lengths not cached: CUDA cores
     (2, 4, 2, 50, 96, [49, 3], None),              # d=96: CUDA-core path
     (2, 3, 1, 50, 32, [16, 49], 5),                # d=32, odd group
+    (2, 8, 2, 300, 64, [299, 5], None),            # r=4, d=64 (transposed products)
+    (1, 48, 2, 400, 128, [399], 200),              # r=24: sub-lanes of 16 and 8 heads
 ]
 
 

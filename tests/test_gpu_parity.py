@@ -228,6 +228,13 @@ DECODE_EDGES = [
     (2, 4, 2, 50, 96, [50, 3], None),
     (2, 3, 1, 50, 32, [17, 50], 5),
     (4200, 2, 1, 3, 128, [b % 4 for b in range(4200)], None),  # lengths read from global memory
+    # groups of up to 8 heads take the transposed products (cache rows as the
+    # MMA's rows): padded head columns, d = 64, windows, partial stages
+    (2, 6, 1, 333, 64, [333, 17], None),          # r=6: 8 columns, 6 heads
+    (3, 10, 2, 257, 128, [257, 113, 0], 100),     # r=5, window, an empty row
+    (2, 4, 2, 500, 64, [500, 250], 64),           # r=2, d=64, window
+    (2, 12, 4, 200, 64, [200, 199], None),        # r=3: 4 columns, 3 heads
+    (1, 14, 2, 1000, 128, [1000], None),          # r=7
 ]
 
 
