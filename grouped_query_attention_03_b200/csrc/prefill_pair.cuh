@@ -197,10 +197,18 @@ __device__ __forceinline__ void softmax_head(const Params &p, Bars &bars, unsign
     // O and P are free here: S(j) was committed after P V(j-1) by the same
     // thread, so S(j) being ready means P V(j-1) has completed.
     if (edge) {
+      // key kb + i is permitted for lo_t - kb <= i <= t - kb.  Most rows of an
+      // edge tile need only the upper bound (the diagonal), and a warp none of
+      // whose rows cuts this tile's keys skips the loop.
+      const int hi_i = t - kb, lo_i = lo_t - kb;
+      if (__any_sync(0xffffffffu, lo_i > 0)) {
 #pragma unroll
-      for (int i = 0; i < kBN; ++i) {
-        const int key = kb + i;
-        if (!(key <= t && key >= lo_t)) s[i] = -INFINITY;
+        for (int i = 0; i < kBN; ++i)
+          if (i > hi_i || i < lo_i) s[i] = -INFINITY;
+      } else if (__any_sync(0xffffffffu, hi_i < kBN - 1)) {
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (i > hi_i) s[i] = -INFINITY;
       }
     }
     // row maximum of s*scale (sc*max(s) for sc > 0, sc*min(s) otherwise)

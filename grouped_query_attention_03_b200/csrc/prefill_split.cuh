@@ -262,10 +262,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tmem_wait_ld();
       const bool edge = (kb + 63 > a0) || (kb < lo_max);
       if (edge) {
+        // key kb + i is permitted for lo_t - kb <= i <= t - kb.  Most rows of an
+        // edge tile need only the upper bound (the diagonal), and a warp none of
+        // whose rows cuts this half's keys skips the loop.
+        const int hi_i = t - kb, lo_i = lo_t - kb;
+        if (__any_sync(0xffffffffu, lo_i > 0)) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = kb + c;
-          if (key > t || key < lo_t) s[c] = -INFINITY;
+          for (int i = 0; i < 64; ++i)
+            if (i > hi_i || i < lo_i) s[i] = -INFINITY;
+        } else if (__any_sync(0xffffffffu, hi_i < 64 - 1)) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (i > hi_i) s[i] = -INFINITY;
         }
       }
       // this half's maximum of s*scale (sc*max(s) for sc > 0, sc*min(s) otherwise)
