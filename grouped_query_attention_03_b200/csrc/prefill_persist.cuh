@@ -496,6 +496,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t idO = tc::idesc_bf16_f32(kBM, D, 0, 1);
         int ai = 0, tcg = 0;
         bool issued = false;
+        bool s0_ahead = false;  // the current item's first S was issued ahead
+        // S of global tile tg from Q buffer qbuf (and Q released after the
+        // item's last S).
+        auto issue_s = [&](int tg, int qbuf, bool last) -> bool {
+          const int sb = tg & 1, ks = tg % K::STAGES;
+          if (!mbar_wait(&bars.k_full[ks], (tg / K::STAGES) & 1, &failed)) return false;
+          tc::fence_after_sync();
+          const uint32_t sQ = smem_u32(smem + K::OFF_Q + qbuf * K::TILE);
+          const uint32_t sK = smem_u32(smem + K::OFF_K + ks * K::TILE);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t off = (k >> 2) * K::BLK + (k & 3) * 32;
+            tc::mma_bf16_ss(tmem + sb * kBN, tc::sw128_desc(sQ + off, 16, 1024),
+                            tc::sw128_desc(sK + off, 16, 1024), idS, k > 0 ? 1u : 0u);
+          }
+          issued = true;
+          tc::mma_commit(&bars.s_full[sb]);
+          if (last) tc::mma_commit(&bars.q_empty[qbuf]);  // Q read by its last S
+          return true;
+        };
         for (int r = 0; r * G < p.n_items && !failed; ++r) {
           const int it = item_of(c, r, G, p.n_items);
           if (it < 0) continue;
@@ -527,25 +547,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::mma_commit(&bars.pv_done[s]);
             return true;
           };
-          if (!mbar_wait(&bars.q_full[qb], (ai / K::NQ) & 1, &failed)) break;
-          const uint32_t sQ = smem_u32(smem + K::OFF_Q + qb * K::TILE);
+          // (a Q wait of a phase already consumed ahead would be ambiguous)
+          if (!s0_ahead && !mbar_wait(&bars.q_full[qb], (ai / K::NQ) & 1, &failed)) break;
           bool ok = true;
           for (int j = 0; j < x.nt; ++j) {
             // S(j) overwrites P of the tile two back, whose P V came first.
-            const int tg = tcg + j, sb = tg & 1, ks = tg % K::STAGES;
-            if (!mbar_wait(&bars.k_full[ks], (tg / K::STAGES) & 1, &failed)) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint32_t sK = smem_u32(smem + K::OFF_K + ks * K::TILE);
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint32_t off = (k >> 2) * K::BLK + (k & 3) * 32;
-              tc::mma_bf16_ss(tmem + sb * kBN, tc::sw128_desc(sQ + off, 16, 1024),
-                              tc::sw128_desc(sK + off, 16, 1024), idS, k > 0 ? 1u : 0u);
-            }
-            issued = true;
-            tc::mma_commit(&bars.s_full[sb]);
-            if (j == x.nt - 1) tc::mma_commit(&bars.q_empty[qb]);  // Q read by its last S
+            if (!(j == 0 && s0_ahead) && !issue_s(tcg + j, qb, j == x.nt - 1)) { ok = false; break; }
             if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+          }
+          // The next item's first S goes ahead of this item's last P V (its
+          // S buffer held P of this item's last tile but one, already read),
+          // so that the softmax does not wait for both at the item boundary.
+          s0_ahead = false;
+          for (int r2 = r + 1; ok && r2 * G < p.n_items; ++r2) {
+            const int it2 = item_of(c, r2, G, p.n_items);
+            if (it2 < 0) continue;
+            const Item x2 = decode_item(p, it2);
+            if (x2.nt == 0) continue;
+            const int qb2 = (ai + 1) % K::NQ;
+            ok = mbar_wait(&bars.q_full[qb2], ((ai + 1) / K::NQ) & 1, &failed) &&
+                 issue_s(tcg + x.nt, qb2, x2.nt == 1);
+            s0_ahead = ok;
+            break;
           }
           if (!ok || !issue_pv(x.nt - 1)) break;
           tc::mma_commit(&bars.o_done[ob]);
