@@ -169,9 +169,9 @@ def pass_stats(ms):
 DECODE_SOURCES = ["decode_splitk.cuh", "common.cuh", "tc_ptx.cuh"]
 DECODE_SHA = "f5815f28d2eec9e95b0d4534fc3a003f3b7bcf1c684160196fa61561e521d95b"
 PAIR_SOURCES = ["prefill_pair.cuh", "common.cuh", "tc_ptx.cuh"]
-PAIR_SHA = "ccbbdc5d3860c03427642dfeab5c45eab3e4763a1b456fb20d8a743e2a3ace59"
+PAIR_SHA = "b55fbb607750b596aa7e864859eb103b7cdf4955fb5bdd52daec85227937995e"
 PERSIST_SOURCES = ["prefill_persist.cuh", "common.cuh", "tc_ptx.cuh"]
-PERSIST_SHA = "18ab7f655a08bbee094ebf3a12788f9f826b987aaea6f4c00b9eff2a8c749338"
+PERSIST_SHA = "914d32926d329e3c21c2ce75b7f79d52bc53e403126ff2afbf4fb0ab7a1907b0"
 CAPTURED_TRAFFIC = [
     {"workload": "decode_b8_n8000", "phase": "decode", "window": None, "hkv": None,
      "bytes": 268_040_448, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
@@ -182,13 +182,13 @@ CAPTURED_TRAFFIC = [
     {"workload": "swa_t32768", "phase": "decode", "window": None, "hkv": None,
      "bytes": 17_117_952, "sources": DECODE_SOURCES, "sha256": DECODE_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": None, "hkv": None,
-     "bytes": 6_356_736, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
+     "bytes": 6_359_808, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
     {"workload": "prefill_b4_t1024", "phase": "prefill", "window": 256, "hkv": None,
-     "bytes": 6_352_896, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 6_356_480, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": None,
-     "bytes": 699_909_888, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
+     "bytes": 688_172_544, "sources": PAIR_SOURCES, "sha256": PAIR_SHA},
     {"workload": "swa_t32768", "phase": "prefill", "window": 4096, "hkv": 32,
-     "bytes": 1_055_563_264, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
+     "bytes": 1_057_996_800, "sources": PERSIST_SOURCES, "sha256": PERSIST_SHA},
 ]
 
 
